@@ -1,0 +1,11 @@
+"""Block-sparse video attention for B200 (sm_100a): fused QK-RMSNorm + 3D RoPE,
+SubBlock block selection and block-sparse attention, behind a C ABI
+(include/sbattn.h) with a thin torch binding."""
+
+from .api import (AttentionLayer, SBAttnError, attention_flops, forward, keep_count, nblocks,  # noqa: F401
+                  qk_norm_rope, select_blocks, select_blocks_pooled, select_blocks_threshold,
+                  select_workspace_bytes)
+
+__all__ = ["AttentionLayer", "SBAttnError", "attention_flops", "forward", "keep_count", "nblocks",
+           "qk_norm_rope", "select_blocks", "select_blocks_pooled", "select_blocks_threshold",
+           "select_workspace_bytes"]

@@ -1,0 +1,262 @@
+"""Python binding of the C ABI (include/sbattn.h) for torch tensors.
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels, on the current torch stream.  torch provides device memory and
+streams.  Tensors must be CUDA, contiguous, [B, N, H, 128] bfloat16 (index
+tensors int32).
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from ._lib import lib, strerror
+
+BLOCK = 64
+HEAD_DIM = 128
+
+
+class SBAttnError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {strerror(code)} (status {code})")
+        self.code = code
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(fn: str, rc: int):
+    if rc != 0:
+        raise SBAttnError(fn, rc)
+
+
+def _act(name, t, dtype=torch.bfloat16):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def nblocks(N: int) -> int:
+    return -(-N // BLOCK)
+
+
+def keep_count(nblk: int, sparsity: float) -> int:
+    """Kept key blocks per query block, diagonal included (host only)."""
+    out = ctypes.c_int(0)
+    _check("sbattn_keep_count", lib().sbattn_keep_count(int(nblk), float(sparsity), ctypes.byref(out)))
+    return out.value
+
+
+def qk_norm_rope(q, k, w_q, w_k, grid, *, dims=(32, 48, 48), theta=10000.0, eps=1e-6,
+                 q_out=None, k_out=None, pool=False):
+    """Fused QK-RMSNorm + 3D RoPE.  grid = (T, Hh, W) with N = T*Hh*W.
+
+    Returns (q_rot, k_rot) or, with pool=True, (q_rot, k_rot, q_bar, k_bar)
+    where the last two are the fp32 [B, H, nblk, d] block means."""
+    _act("q", q), _act("k", k), _act("w_q", w_q), _act("w_k", w_k)
+    B, N, H, d = q.shape
+    T, Hh, W = grid
+    q_out = torch.empty_like(q) if q_out is None else _act("q_out", q_out)
+    k_out = torch.empty_like(k) if k_out is None else _act("k_out", k_out)
+    q_bar = k_bar = None
+    if pool:
+        q_bar = torch.empty((B, H, nblocks(N), d), device=q.device, dtype=torch.float32)
+        k_bar = torch.empty_like(q_bar)
+    rc = lib().sbattn_qk_norm_rope(_ptr(q), _ptr(k), _ptr(w_q), _ptr(w_k), _ptr(q_out), _ptr(k_out),
+                                   _ptr(q_bar), _ptr(k_bar), B, T, Hh, W, H, d, dims[0], dims[1], dims[2],
+                                   float(theta), float(eps), _stream(q.device))
+    _check("sbattn_qk_norm_rope", rc)
+    return (q_out, k_out, q_bar, k_bar) if pool else (q_out, k_out)
+
+
+def select_workspace_bytes(B, N, H, d=HEAD_DIM) -> int:
+    return lib().sbattn_select_workspace_bytes(B, N, H, d)
+
+
+def _select_outputs(B, H, nblk, cap, device, want_scores):
+    kept_idx = torch.empty((B, H, nblk, cap), device=device, dtype=torch.int32)
+    kept_cnt = torch.empty((B, H, nblk), device=device, dtype=torch.int32)
+    scores = torch.empty((B, H, nblk, nblk), device=device, dtype=torch.float32) if want_scores else None
+    return kept_idx, kept_cnt, scores
+
+
+def select_blocks(q_rot, k_rot, sparsity, *, return_scores=False, workspace=None, capacity=None):
+    """SubBlock selection (budget form) from rotated Q/K.
+    Returns (kept_idx [B,H,nblk,K], kept_cnt [B,H,nblk]) (+ scores)."""
+    _act("q_rot", q_rot), _act("k_rot", k_rot)
+    B, N, H, d = q_rot.shape
+    nblk = nblocks(N)
+    K = keep_count(nblk, sparsity)
+    cap = K if capacity is None else capacity
+    kept_idx, kept_cnt, scores = _select_outputs(B, H, nblk, cap, q_rot.device, return_scores)
+    need = select_workspace_bytes(B, N, H, d)
+    if workspace is None:
+        workspace = torch.empty(need, device=q_rot.device, dtype=torch.uint8)
+    rc = lib().sbattn_select_blocks(_ptr(q_rot), _ptr(k_rot), B, N, H, d, float(sparsity), _ptr(kept_idx),
+                                    _ptr(kept_cnt), cap, _ptr(scores), _ptr(workspace), workspace.numel(),
+                                    _stream(q_rot.device))
+    _check("sbattn_select_blocks", rc)
+    return (kept_idx, kept_cnt, scores) if return_scores else (kept_idx, kept_cnt)
+
+
+def select_blocks_pooled(q_bar, k_bar, sparsity, *, return_scores=False, capacity=None):
+    """Budget selection from pooled fp32 [B, H, nblk, d] block means."""
+    _act("q_bar", q_bar, torch.float32), _act("k_bar", k_bar, torch.float32)
+    B, H, nblk, d = q_bar.shape
+    K = keep_count(nblk, sparsity)
+    cap = K if capacity is None else capacity
+    kept_idx, kept_cnt, scores = _select_outputs(B, H, nblk, cap, q_bar.device, return_scores)
+    rc = lib().sbattn_select_blocks_pooled(_ptr(q_bar), _ptr(k_bar), B, nblk, H, d, float(sparsity),
+                                           _ptr(kept_idx), _ptr(kept_cnt), cap, _ptr(scores),
+                                           _stream(q_bar.device))
+    _check("sbattn_select_blocks_pooled", rc)
+    return (kept_idx, kept_cnt, scores) if return_scores else (kept_idx, kept_cnt)
+
+
+def select_blocks_threshold(q_bar, k_bar, tau, *, return_scores=False):
+    """Threshold selection: the diagonal plus every block with score >= tau."""
+    _act("q_bar", q_bar, torch.float32), _act("k_bar", k_bar, torch.float32)
+    B, H, nblk, d = q_bar.shape
+    kept_idx, kept_cnt, scores = _select_outputs(B, H, nblk, nblk, q_bar.device, return_scores)
+    rc = lib().sbattn_select_blocks_threshold(_ptr(q_bar), _ptr(k_bar), B, nblk, H, d, float(tau),
+                                              _ptr(kept_idx), _ptr(kept_cnt), nblk, _ptr(scores),
+                                              _stream(q_bar.device))
+    _check("sbattn_select_blocks_threshold", rc)
+    return (kept_idx, kept_cnt, scores) if return_scores else (kept_idx, kept_cnt)
+
+
+def forward(q_rot, k_rot, v, kept_idx, kept_cnt, *, scale=None, out=None, status=None):
+    """Block-sparse attention over the kept key blocks; returns out [B,N,H,d] bf16.
+
+    status: optional int32 CUDA tensor of one element; device-side errors are
+    recorded there (it is not cleared by the call)."""
+    _act("q_rot", q_rot), _act("k_rot", k_rot), _act("v", v)
+    _act("kept_idx", kept_idx, torch.int32), _act("kept_cnt", kept_cnt, torch.int32)
+    B, N, H, d = q_rot.shape
+    out = torch.empty_like(q_rot) if out is None else _act("out", out)
+    if status is not None:
+        _act("status", status, torch.int32)
+    rc = lib().sbattn_forward(_ptr(q_rot), _ptr(k_rot), _ptr(v), _ptr(kept_idx), _ptr(kept_cnt),
+                              kept_idx.shape[-1], _ptr(out), B, N, H, d,
+                              0.0 if scale is None else float(scale), _ptr(status), _stream(q_rot.device))
+    _check("sbattn_forward", rc)
+    return out
+
+
+class AttentionLayer:
+    """The whole hot path of one attention layer with preallocated device
+    buffers: prologue (with fused block pooling) -> selection -> attention.
+
+    `__call__` takes device or host tensors; host tensors are copied in (and
+    the output copied back) on the current stream, which is what an
+    end-to-end caller with host buffers pays.
+    """
+
+    def __init__(self, B, T, Hh, W, H, sparsity, *, device="cuda", dims=(32, 48, 48), theta=10000.0,
+                 eps=1e-6, fused_pool=True):
+        self.B, self.T, self.Hh, self.W, self.H = B, T, Hh, W, H
+        self.N = T * Hh * W
+        self.nblk = nblocks(self.N)
+        self.sparsity, self.dims, self.theta, self.eps = sparsity, dims, theta, eps
+        self.fused_pool = fused_pool
+        self.K = keep_count(self.nblk, sparsity)
+        dev = torch.device(device)
+        shp = (B, self.N, H, HEAD_DIM)
+        self.dev = dev
+        self.q_in = torch.empty(shp, device=dev, dtype=torch.bfloat16)
+        self.k_in = torch.empty_like(self.q_in)
+        self.v_in = torch.empty_like(self.q_in)
+        self.wq_in = torch.empty((HEAD_DIM,), device=dev, dtype=torch.bfloat16)
+        self.wk_in = torch.empty_like(self.wq_in)
+        self.q_rot = torch.empty_like(self.q_in)
+        self.k_rot = torch.empty_like(self.q_in)
+        self.out = torch.empty_like(self.q_in)
+        self.q_bar = torch.empty((B, H, self.nblk, HEAD_DIM), device=dev, dtype=torch.float32)
+        self.k_bar = torch.empty_like(self.q_bar)
+        self.kept_idx = torch.empty((B, H, self.nblk, self.K), device=dev, dtype=torch.int32)
+        self.kept_cnt = torch.empty((B, H, self.nblk), device=dev, dtype=torch.int32)
+        self.status = torch.zeros((1,), device=dev, dtype=torch.int32)
+        self.workspace = None if fused_pool else torch.empty(
+            select_workspace_bytes(B, self.N, H), device=dev, dtype=torch.uint8)
+
+    def run_device(self, q, k, v, w_q, w_k, events=None):
+        """Run the path on device tensors already resident in HBM.
+
+        events: optional 4 CUDA events, recorded on the launching stream
+        before the prologue, before the selection, before the attention and
+        after it (per-kernel device timing)."""
+        L, s = lib(), _stream(self.dev)
+        B, N, H, d = self.B, self.N, self.H, HEAD_DIM
+        if events is not None:
+            events[0].record()
+        if self.fused_pool:
+            rc = L.sbattn_qk_norm_rope(_ptr(q), _ptr(k), _ptr(w_q), _ptr(w_k), _ptr(self.q_rot), _ptr(self.k_rot),
+                                       _ptr(self.q_bar), _ptr(self.k_bar), B, self.T, self.Hh, self.W, H, d,
+                                       *self.dims, float(self.theta), float(self.eps), s)
+            _check("sbattn_qk_norm_rope", rc)
+            if events is not None:
+                events[1].record()
+            rc = L.sbattn_select_blocks_pooled(_ptr(self.q_bar), _ptr(self.k_bar), B, self.nblk, H, d,
+                                               float(self.sparsity), _ptr(self.kept_idx), _ptr(self.kept_cnt),
+                                               self.K, None, s)
+            _check("sbattn_select_blocks_pooled", rc)
+        else:
+            rc = L.sbattn_qk_norm_rope(_ptr(q), _ptr(k), _ptr(w_q), _ptr(w_k), _ptr(self.q_rot), _ptr(self.k_rot),
+                                       None, None, B, self.T, self.Hh, self.W, H, d,
+                                       *self.dims, float(self.theta), float(self.eps), s)
+            _check("sbattn_qk_norm_rope", rc)
+            if events is not None:
+                events[1].record()
+            rc = L.sbattn_select_blocks(_ptr(self.q_rot), _ptr(self.k_rot), B, N, H, d, float(self.sparsity),
+                                        _ptr(self.kept_idx), _ptr(self.kept_cnt), self.K, None,
+                                        _ptr(self.workspace), self.workspace.numel(), s)
+            _check("sbattn_select_blocks", rc)
+        if events is not None:
+            events[2].record()
+        rc = L.sbattn_forward(_ptr(self.q_rot), _ptr(self.k_rot), _ptr(v), _ptr(self.kept_idx),
+                              _ptr(self.kept_cnt), self.K, _ptr(self.out), B, N, H, d, 0.0,
+                              _ptr(self.status), s)
+        _check("sbattn_forward", rc)
+        if events is not None:
+            events[3].record()
+        return self.out
+
+    # kernels launched per run_device call (prologue, selection [+ pooling], attention)
+    @property
+    def launches_per_call(self) -> int:
+        return 3 if self.fused_pool else 4
+
+    def __call__(self, q, k, v, w_q, w_k, out_host=None):
+        if q.is_cuda:
+            return self.run_device(q, k, v, w_q, w_k)
+        for dst, src in ((self.q_in, q), (self.k_in, k), (self.v_in, v), (self.wq_in, w_q), (self.wk_in, w_k)):
+            dst.copy_(src, non_blocking=True)
+        o = self.run_device(self.q_in, self.k_in, self.v_in, self.wq_in, self.wk_in)
+        if out_host is None:
+            out_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        out_host.copy_(o, non_blocking=True)
+        return out_host
+
+    def check_status(self):
+        """Synchronise and raise if a kernel recorded a device-side error."""
+        code = int(self.status.item())
+        if code != 0:
+            raise SBAttnError("device status", code)
+
+
+def attention_flops(B, N, H, K, d=HEAD_DIM) -> float:
+    """Effective FLOPs of the attention over the kept blocks: 4 * N * (64 K) * d
+    per (batch, head) -- QK^T and PV at two flops per multiply-add, 64 keys per
+    kept block."""
+    return 4.0 * B * H * N * (BLOCK * K) * d

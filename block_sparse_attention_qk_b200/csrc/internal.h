@@ -1,0 +1,63 @@
+// Launcher interface between the C ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace sbattn {
+
+struct PrologueArgs {
+  const uint16_t* q;   // input rows (prologue: raw Q; pooling: rotated Q)
+  const uint16_t* k;
+  const uint16_t* w_q;
+  const uint16_t* w_k;
+  uint16_t* q_out;
+  uint16_t* k_out;
+  float* q_pool;       // [B, H, nblk, d] or null
+  float* k_pool;
+  int B, N, H, T, Hh, W, nblk;
+  int dim_t, dim_h, dim_w;
+  float theta, eps;
+};
+
+// Largest rotation table the prologue keeps in shared memory.
+constexpr size_t kMaxRopeTableBytes = 160 * 1024;
+size_t prologue_table_bytes(int T, int Hh, int W, int dim_t, int dim_h, int dim_w);
+int launch_prologue(const PrologueArgs& a, cudaStream_t stream);
+int launch_pool(const PrologueArgs& a, cudaStream_t stream);
+
+struct SelectArgs {
+  const float* q_bar;  // [B, H, nblk, d]
+  const float* k_bar;
+  int B, H, nblk;
+  int keep;            // budget form: kept blocks per row (diagonal included)
+  int threshold_mode;  // 1: keep score >= tau instead of a budget
+  float tau;
+  int32_t* kept_idx;   // [B, H, nblk, K_capacity]
+  int32_t* kept_cnt;   // [B, H, nblk]
+  int K_capacity;
+  float* scores;       // [B, H, nblk, nblk] or null
+};
+
+// Largest nblk the selection kernel handles (one score row in shared memory).
+int select_max_nblk();
+int launch_select(const SelectArgs& a, cudaStream_t stream);
+
+struct AttentionArgs {
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  const int32_t* kept_idx;
+  const int32_t* kept_cnt;
+  uint16_t* out;
+  int32_t* status;
+  int B, N, H, nblk, K_capacity;
+  float scale;
+};
+
+int launch_attention(const AttentionArgs& a, cudaStream_t stream);
+
+// TMA descriptor of a [B, N, H, 128] bf16 tensor (box: 64 channels x 64 tokens
+// of one head, 128-byte swizzle, zero fill past N).
+int make_bf16_row_map(CUtensorMap* map, const void* base, int B, int N, int H);
+
+}  // namespace sbattn

@@ -1,0 +1,191 @@
+/*
+ * sbattn.h -- C ABI of the block-sparse video attention library (sm_100a).
+ *
+ * The library computes one video-DiT attention layer's hot path:
+ *   1. sbattn_qk_norm_rope    fused per-head QK-RMSNorm + 3D RoPE;
+ *   2. sbattn_select_blocks   SubBlock block selection: 64-token blocks,
+ *                             mean-pooled block scores, per query block the
+ *                             diagonal key block plus the top-scoring ones;
+ *   3. sbattn_forward         attention over the kept key blocks only.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [p3] xiaodao.ai "MiniMax-H3 的 6.24 倍，不能直接算成六倍产能":
+ *        section "先把近两倍的免费收益拿走" -- fused QK RMSNorm and 3D RoPE
+ *        kernel, fewer intermediate tensors, memory traffic and launches;
+ *        section "6.24 倍里，真正有损的部分大约是三倍" -- SubBlock cuts query
+ *        and key into 64-token blocks, estimates which key blocks contribute
+ *        little and keeps only the high-scoring ones for a block-sparse
+ *        attention kernel; sparsity 0.75 keeps about a quarter.
+ *   [p4] chat-gpts.plus "MiniMax-H3 在 8×H200 上基准测试：无损加速 1.95×，
+ *        最高 6.24×（SSIM 0.76-0.91）", section "事件核心：发生了什么" --
+ *        SubBlock skips attention blocks below a threshold.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Activations are bfloat16 bit patterns (uint16_t), contiguous, laid out
+ *    [B, N, H, d] (batch, token, head, channel; channel fastest), the layout a
+ *    fused QKV projection writes and the output projection reads.
+ *  - d must be 128.  N is the token count; tokens are cut into nblk =
+ *    ceil(N / 64) blocks of 64 (the last one may be partial).
+ *  - All tensor pointers are DEVICE pointers owned by the caller and must be
+ *    16-byte aligned.  The library allocates and frees nothing, keeps no state
+ *    between calls, never synchronises, and launches only on `stream`
+ *    (a cudaStream_t passed as void*; NULL means the legacy default stream).
+ *  - Every call returns an int status (SBATTN_OK on success).  Argument
+ *    errors are detected on the host before anything is launched; a call that
+ *    returns an error has launched nothing.  SBATTN_ERR_CUDA reports a launch
+ *    failure (cudaGetLastError after the launch).
+ *  - Calls are asynchronous: results are ready once the stream reaches them.
+ */
+#ifndef SBATTN_H
+#define SBATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SBATTN_API __attribute__((visibility("default")))
+#else
+#define SBATTN_API
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define SBATTN_OK                    0
+#define SBATTN_ERR_INVALID_ARG       1  /* null pointer, negative size, bad number */
+#define SBATTN_ERR_UNSUPPORTED_SHAPE 2  /* d != 128, N != T*Hh*W, bad RoPE split, too large */
+#define SBATTN_ERR_MISALIGNED        3  /* a tensor pointer is not 16-byte aligned */
+#define SBATTN_ERR_WORKSPACE         4  /* workspace missing or too small */
+#define SBATTN_ERR_CUDA              5  /* CUDA runtime error at launch */
+#define SBATTN_ERR_DEVICE            6  /* a device-side check failed (see status word) */
+#define SBATTN_ERR_TIMEOUT           7  /* a bounded wait inside a kernel ran out */
+#define SBATTN_ERR_CAPACITY          8  /* kept-list capacity smaller than the budget */
+
+#define SBATTN_BLOCK 64                 /* tokens per block ([p3], "6.24 倍里…") */
+
+/* Human-readable name of a status code (static string, never NULL). */
+SBATTN_API const char* sbattn_strerror(int status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+SBATTN_API int sbattn_version(void);
+
+/* ---- 1. fused QK-RMSNorm + 3D RoPE -------------------------------------
+ * [p3] "先把近两倍的免费收益拿走": QK RMSNorm and 3D RoPE fused in one kernel.
+ *
+ * For every (b, n, h) and X in {Q, K}, with x the d-vector of that row:
+ *     r = 1 / sqrt(mean_c(x_c^2) + eps);   y = x * r * w_X   (w_X: [d])
+ * then the 3D rotary embedding: token n of the T x Hh x W latent grid sits at
+ * t = n / (Hh*W), h = (n / W) % Hh, w = n % W; channels [0, dim_t) rotate with
+ * t, [dim_t, dim_t+dim_h) with h, the last dim_w with w; inside a section of
+ * size D starting at channel o, the pair (o+2m, o+2m+1) turns by
+ * pos * theta^(-2m/D):  (a, b) -> (a cos - b sin, a sin + b cos).
+ * Arithmetic in fp32, output rounded to bf16 (nearest even).
+ *
+ *   q, k          [B, N, H, d] bf16 input, N = T*Hh*W
+ *   w_q, w_k      [d] bf16 RMSNorm weights (shared by all heads)
+ *   q_out, k_out  [B, N, H, d] bf16 output; may alias q / k (in place)
+ *   dim_t+dim_h+dim_w == d, each even and a multiple of 8
+ *   q_pool, k_pool  optional (may be NULL, both or neither): fp32
+ *                 [B, H, nblk, d] block means of q_out / k_out, i.e. the
+ *                 pooled vectors sbattn_select_blocks_pooled consumes; writing
+ *                 them here saves re-reading q_out / k_out.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (d != 128, bad split, grid whose
+ * rotation table exceeds 160 KiB), MISALIGNED, CUDA.
+ */
+SBATTN_API int sbattn_qk_norm_rope(const uint16_t* q, const uint16_t* k,
+                                   const uint16_t* w_q, const uint16_t* w_k,
+                                   uint16_t* q_out, uint16_t* k_out,
+                                   float* q_pool, float* k_pool,
+                                   int B, int T, int Hh, int W, int H, int d,
+                                   int dim_t, int dim_h, int dim_w,
+                                   float theta, float eps, void* stream);
+
+/* ---- 2. block selection (SubBlock, budget form) -------------------------
+ * [p3] "6.24 倍里，真正有损的部分大约是三倍".
+ *
+ * Kept blocks per query block: K = ceil((1 - s) * nblk), with s read as a
+ * decimal of at most six fractional digits (s_micro = llround(s * 1e6);
+ * K = ceil((1e6 - s_micro) * nblk / 1e6) in exact integer arithmetic),
+ * clamped to [1, nblk].  Rejects s outside [0, 1] or NaN with INVALID_ARG.
+ * Host-only; needs no GPU.
+ */
+SBATTN_API int sbattn_keep_count(int nblk, double sparsity, int* K_out);
+
+/* Workspace bytes sbattn_select_blocks needs: two fp32 [B, H, nblk, d]
+ * pooled tensors (2 * B*H*nblk*d*4 bytes).  Returns 0 on invalid sizes. */
+SBATTN_API size_t sbattn_select_workspace_bytes(int B, int N, int H, int d);
+
+/* For every (b, h) and query block i:
+ *   q_bar_i = mean of the (up to) 64 rows of q_rot in block i (k_bar likewise);
+ *   score s_ij = q_bar_i . k_bar_j  (fp32);
+ *   kept(i) = {i} + the K-1 highest-scoring j != i (equal scores: lower j
+ *   first), written sorted ascending.
+ *
+ *   q_rot, k_rot  [B, N, H, d] bf16 (the prologue's output)
+ *   kept_idx      [B, H, nblk, K_capacity] int32 output; row (b,h,i) holds
+ *                 its kept block ids in entries [0, kept_cnt); entries past
+ *                 kept_cnt are set to -1
+ *   kept_cnt      [B, H, nblk] int32 output (= K for every row)
+ *   K_capacity    >= K, else SBATTN_ERR_CAPACITY
+ *   scores        optional fp32 [B, H, nblk, nblk] output of s_ij (NULL to skip)
+ *   workspace     device scratch of >= sbattn_select_workspace_bytes bytes,
+ *                 16-byte aligned; its contents on entry do not matter
+ */
+SBATTN_API int sbattn_select_blocks(const uint16_t* q_rot, const uint16_t* k_rot,
+                                    int B, int N, int H, int d, double sparsity,
+                                    int32_t* kept_idx, int32_t* kept_cnt, int K_capacity,
+                                    float* scores, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
+/* Same selection from already pooled fp32 [B, H, nblk, d] block means (as
+ * written by sbattn_qk_norm_rope's q_pool / k_pool).  No workspace. */
+SBATTN_API int sbattn_select_blocks_pooled(const float* q_bar, const float* k_bar,
+                                           int B, int nblk, int H, int d, double sparsity,
+                                           int32_t* kept_idx, int32_t* kept_cnt, int K_capacity,
+                                           float* scores, void* stream);
+
+/* Threshold form ([p4] "事件核心…": blocks scoring below a threshold are
+ * skipped): kept(i) = {i} + every j != i with s_ij >= tau, sorted ascending;
+ * kept_cnt varies per row (1..nblk); K_capacity must be >= nblk.
+ * Inputs are pooled means as for sbattn_select_blocks_pooled. */
+SBATTN_API int sbattn_select_blocks_threshold(const float* q_bar, const float* k_bar,
+                                              int B, int nblk, int H, int d, float tau,
+                                              int32_t* kept_idx, int32_t* kept_cnt, int K_capacity,
+                                              float* scores, void* stream);
+
+/* ---- 3. block-sparse attention -----------------------------------------
+ * [p3] "6.24 倍里…": only the kept key blocks enter the attention kernel.
+ *
+ * For every (b, h) and query block i with S = tokens of the kept key blocks
+ * kept_idx[b,h,i,0:kept_cnt[b,h,i]]:
+ *     O_i = softmax(Q_i K_S^T * scale) V_S      (non-causal; keys outside S
+ *                                                contribute nothing)
+ * bf16 tensor-core products with fp32 accumulation and an fp32 softmax.
+ *
+ *   q_rot, k_rot, v [B, N, H, d] bf16
+ *   kept_idx        [B, H, nblk, K_capacity] int32, each entry in [0, nblk),
+ *                   no repeats within a row (any order)
+ *   kept_cnt        [B, H, nblk] int32, each in [1, K_capacity]
+ *   out             [B, N, H, d] bf16 output (must not alias the inputs)
+ *   softmax_scale   <= 0 selects 1/sqrt(d)
+ *   status          optional device int32 (may be NULL).  If given, the
+ *                   kernel stores a nonzero SBATTN_ERR_* code there when a
+ *                   kept index or count is out of range (that block/row is
+ *                   skipped) or a bounded internal wait runs out; it never
+ *                   clears it.  Zero it before the call and read it after the
+ *                   stream has reached the call.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (d != 128), MISALIGNED, CUDA.
+ */
+SBATTN_API int sbattn_forward(const uint16_t* q_rot, const uint16_t* k_rot, const uint16_t* v,
+                              const int32_t* kept_idx, const int32_t* kept_cnt, int K_capacity,
+                              uint16_t* out, int B, int N, int H, int d,
+                              float softmax_scale, int32_t* status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SBATTN_H */

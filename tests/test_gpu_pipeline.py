@@ -1,0 +1,99 @@
+"""End-to-end parity of the whole path (prologue -> selection -> attention)
+through the C ABI, against the oracle's own chain from the same raw inputs.
+
+Small workloads are compared in full.  The full-size video workloads run in
+the launch configuration the benchmark times (AttentionLayer with the pooled
+means fused into the prologue) and are compared on sampled heads, query blocks
+and tokens that the oracle computes one by one.
+
+In a chain, the GPU's bf16 prologue output differs from the oracle's rounded
+output in about 0.1 % of elements by one ulp, which can flip a selection at a
+near tie; rows whose kept sets differ are counted (decisions must agree at
+>= 99.9 %) and their attention is not compared, because both answers are
+valid for their own kept set.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_qk_b200 as sb
+from block_sparse_attention_qk_b200.inputs import WORKLOADS, custom_workload, make_inputs
+from oracle import sbattn_oracle as orc
+
+from .parity import check_attention, check_kept_structure, check_prologue, f64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _chain_compare(wl, layer, x_cpu, out, heads, rows_per_head, rng):
+    """Compare a layer run against the oracle chain on the given heads."""
+    K = orc.keep_count(wl.nblk, wl.sparsity)
+    gidx_all = layer.kept_idx.cpu().numpy()
+    gcnt_all = layer.kept_cnt.cpu().numpy()
+    check_kept_structure(gidx_all, gcnt_all, wl.nblk, K)
+    stats = {"rows": 0, "rows_differing": 0, "decisions": 0, "disagree": 0}
+    for b in range(wl.B):
+        for h in heads:
+            sl = lambda t: t[b:b + 1, :, h:h + 1].contiguous()
+            qh, kh, vh = f64(sl(x_cpu["q"])), f64(sl(x_cpu["k"])), f64(sl(x_cpu["v"]))
+            qr, kr = orc.qk_norm_rope(qh, kh, f64(x_cpu["w_q"]), f64(x_cpu["w_k"]), wl.T, wl.Hh, wl.W)
+            check_prologue(f64(layer.q_rot[b:b + 1, :, h:h + 1]), qr, f"q head {h}")
+            check_prologue(f64(layer.k_rot[b:b + 1, :, h:h + 1]), kr, f"k head {h}")
+            qr16, kr16 = orc.round_to_bf16(qr), orc.round_to_bf16(kr)
+            q_bar, k_bar = orc.block_pool(qr16), orc.block_pool(kr16)
+            s = orc.block_scores(q_bar, k_bar)[0, 0]
+            rows = sorted(set([0, wl.nblk - 1]) | set(rng.choice(wl.nblk, size=min(rows_per_head, wl.nblk),
+                                                                   replace=False).tolist()))
+            for i in rows:
+                ref = orc.select_row(s[i], i, K)
+                got = gidx_all[b, h, i, :gcnt_all[b, h, i]]
+                stats["rows"] += 1
+                stats["decisions"] += wl.nblk
+                if set(got.tolist()) != set(ref.tolist()):
+                    stats["rows_differing"] += 1
+                    stats["disagree"] += len(set(got.tolist()) ^ set(ref.tolist()))
+                    continue
+                o_ref = orc.attention_block(qr16, kr16, vh, ref, 0, 0, i)
+                lo, hi = i * 64, min(wl.N, (i + 1) * 64)
+                check_attention(f64(out[b, lo:hi, h]), o_ref, f"attention head {h} block {i}")
+    agree = 1 - stats["disagree"] / stats["decisions"]
+    assert agree >= 0.999, stats
+    return stats
+
+
+@pytest.mark.parametrize("name", ["tiny", "dense", "ragged"])
+def test_chain_small(name):
+    wl = {"tiny": WORKLOADS["tiny"], "dense": WORKLOADS["dense"].with_sparsity(0.75),
+          "ragged": custom_workload("ragged", B=2, H=3, T=3, Hh=7, W=13, sparsity=0.6, seed=21)}[name]
+    x = make_inputs(wl)
+    for fused in (True, False):
+        layer = sb.AttentionLayer(wl.B, wl.T, wl.Hh, wl.W, wl.H, wl.sparsity, device=DEV, fused_pool=fused)
+        out = layer(x["q"].pin_memory(), x["k"].pin_memory(), x["v"].pin_memory(), x["w_q"], x["w_k"])
+        torch.cuda.synchronize()
+        layer.check_status()
+        _chain_compare(wl, layer, x, out, range(wl.H), wl.nblk, np.random.default_rng(0))
+
+
+@pytest.mark.parametrize("name", ["5s", "5s_aggr", "10s", "portrait"])
+def test_full_size_sampled(name):
+    wl = WORKLOADS[name]
+    x = make_inputs(wl, device=DEV)  # full-size draw on the device
+    layer = sb.AttentionLayer(wl.B, wl.T, wl.Hh, wl.W, wl.H, wl.sparsity, device=DEV)
+    out = layer.run_device(x["q"], x["k"], x["v"], x["w_q"], x["w_k"])
+    torch.cuda.synchronize()
+    layer.check_status()
+    rng = np.random.default_rng(123)
+    heads = sorted(rng.choice(wl.H, size=2, replace=False).tolist())
+    x_cpu = {k: (v[:, :, heads].cpu() if v.dim() == 4 else v.cpu()) for k, v in x.items()}
+    out_cpu = out[:, :, heads].cpu()
+
+    class _View:  # the layer's buffers restricted to the sampled heads
+        q_rot = layer.q_rot[:, :, heads].cpu()
+        k_rot = layer.k_rot[:, :, heads].cpu()
+        kept_idx = layer.kept_idx[:, heads].cpu()
+        kept_cnt = layer.kept_cnt[:, heads].cpu()
+
+    stats = _chain_compare(wl, _View, x_cpu, out_cpu, range(len(heads)), 12, rng)
+    assert stats["rows"] >= 2 * 12
