@@ -73,7 +73,8 @@ def test_chain_small(name):
         out = layer(x["q"].pin_memory(), x["k"].pin_memory(), x["v"].pin_memory(), x["w_q"], x["w_k"])
         torch.cuda.synchronize()
         layer.check_status()
-        _chain_compare(wl, layer, x, out, range(wl.H), wl.nblk, np.random.default_rng(0))
+        heads = (2, 7) if name == "dense" else range(wl.H)  # fp64 cost: two of the dense check's 8 heads
+        _chain_compare(wl, layer, x, out, heads, wl.nblk, np.random.default_rng(0))
 
 
 @pytest.mark.parametrize("name", ["5s", "5s_aggr", "10s", "portrait"])
