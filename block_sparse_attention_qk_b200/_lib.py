@@ -24,6 +24,8 @@ SIGNATURES = {
                                              _c_void, _c_void, _c_int, _c_void, _c_void]),
     "sbattn_select_blocks_threshold": (_c_int, [_c_void, _c_void, _c_int, _c_int, _c_int, _c_int, _c_float,
                                                 _c_void, _c_void, _c_int, _c_void, _c_void]),
+    "sbattn_select_blocks_noalloc": (_c_int, [_c_void, _c_void, _c_int, _c_int, _c_int, _c_int, _c_double,
+                                              _c_void, _c_void, _c_int, _c_void, _c_void]),
     "sbattn_forward": (_c_int, [_c_void, _c_void, _c_void, _c_void, _c_void, _c_int, _c_void,
                                 _c_int, _c_int, _c_int, _c_int, _c_float, _c_void, _c_void]),
 }

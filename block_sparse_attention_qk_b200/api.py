@@ -110,6 +110,22 @@ def select_blocks(q_rot, k_rot, sparsity, *, return_scores=False, workspace=None
     return (kept_idx, kept_cnt, scores) if return_scores else (kept_idx, kept_cnt)
 
 
+def select_blocks_noalloc(q_rot, k_rot, sparsity, *, return_scores=False, capacity=None):
+    """select_blocks without a workspace: the pooled means use the library's
+    built-in scratch array (for callers that cannot allocate device memory;
+    limited to B * H * nblk <= 4096; calls that overlap on the GPU race)."""
+    _act("q_rot", q_rot), _act("k_rot", k_rot)
+    B, N, H, d = q_rot.shape
+    nblk = nblocks(N)
+    K = keep_count(nblk, sparsity)
+    cap = K if capacity is None else capacity
+    kept_idx, kept_cnt, scores = _select_outputs(B, H, nblk, cap, q_rot.device, return_scores)
+    rc = lib().sbattn_select_blocks_noalloc(_ptr(q_rot), _ptr(k_rot), B, N, H, d, float(sparsity), _ptr(kept_idx),
+                                            _ptr(kept_cnt), cap, _ptr(scores), _stream(q_rot.device))
+    _check("sbattn_select_blocks_noalloc", rc)
+    return (kept_idx, kept_cnt, scores) if return_scores else (kept_idx, kept_cnt)
+
+
 def select_blocks_pooled(q_bar, k_bar, sparsity, *, return_scores=False, capacity=None):
     """Budget selection from pooled fp32 [B, H, nblk, d] block means."""
     _act("q_bar", q_bar, torch.float32), _act("k_bar", k_bar, torch.float32)

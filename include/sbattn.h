@@ -156,6 +156,34 @@ SBATTN_API int sbattn_select_blocks_threshold(const float* q_bar, const float* k
                                               int32_t* kept_idx, int32_t* kept_cnt, int K_capacity,
                                               float* scores, void* stream);
 
+/* Same selection as sbattn_select_blocks, for callers that cannot allocate
+ * device memory when they run the layer -- a plugin-style host that passes
+ * the library only the layer's inputs and outputs and owns all other device
+ * memory, or a runtime that plans its memory up front and forbids allocation
+ * once serving.  The pages have no counterpart to this call; it exists only
+ * for such callers.
+ *
+ * The pooled block means live in a fixed scratch array compiled into the
+ * library (4 MiB of device memory, held on every GPU that loads the library
+ * until the process exits), so the call allocates nothing and takes no
+ * workspace.  Limit: B * H * ceil(N/64) <= SBATTN_NOALLOC_MAX_POOLED_ROWS;
+ * larger problems are rejected with SBATTN_ERR_WORKSPACE before anything is
+ * launched (use sbattn_select_blocks with a workspace for them).
+ *
+ * The first call on each device looks up that device's address of the
+ * scratch array (with that device current); make that first call before any
+ * stream capture.  All calls on a device share the one array and each call
+ * overwrites every value it reads, so nothing needs clearing between calls;
+ * but calls whose work overlaps on the GPU (different streams, or different
+ * host threads, without ordering between them) race on it.
+ * Other arguments, outputs and errors as for sbattn_select_blocks.
+ */
+#define SBATTN_NOALLOC_MAX_POOLED_ROWS 4096
+SBATTN_API int sbattn_select_blocks_noalloc(const uint16_t* q_rot, const uint16_t* k_rot,
+                                            int B, int N, int H, int d, double sparsity,
+                                            int32_t* kept_idx, int32_t* kept_cnt, int K_capacity,
+                                            float* scores, void* stream);
+
 /* ---- 3. block-sparse attention -----------------------------------------
  * [p3] "6.24 倍里…": only the kept key blocks enter the attention kernel.
  *
