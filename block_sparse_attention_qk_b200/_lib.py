@@ -7,7 +7,6 @@ from __future__ import annotations
 import ctypes
 import os
 
-from . import build as _build
 
 _c_int, _c_double, _c_float, _c_size, _c_void = ctypes.c_int, ctypes.c_double, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p
 
@@ -34,7 +33,9 @@ _LIB = None
 
 
 def lib_path() -> str:
-    return _build.LIB_PATH
+    from .build import LIB_PATH
+
+    return LIB_PATH
 
 
 def lib() -> ctypes.CDLL:

@@ -48,19 +48,24 @@ struct RopeTable {
 template <bool kNormRope, bool kPool>
 __global__ void __launch_bounds__(kThreads) prologue_kernel(PrologueArgs a, RopeTable rt) {
   extern __shared__ float2 tab[];
+  __shared__ double inv_freq[kHeadDim / 2];  // theta^(-2m/D) per section pair
 
   if constexpr (kNormRope) {
+    for (int p = threadIdx.x; p < kHeadDim / 2; p += kThreads) {
+      const int axis = p < rt.half[0] ? 0 : (p < rt.half[0] + rt.half[1] ? 1 : 2);
+      const int m = p - (axis > 0 ? rt.half[0] : 0) - (axis > 1 ? rt.half[1] : 0);
+      inv_freq[p] = pow((double)a.theta, -(2.0 * m) / (2.0 * rt.half[axis]));
+    }
+    __syncthreads();
     for (int e = threadIdx.x; e < rt.entries; e += kThreads) {
-      int axis = (e >= rt.off[2]) ? 2 : (e >= rt.off[1]) ? 1 : 0;
-      int local = e - rt.off[axis];
-      int pos = local / rt.half[axis];
-      int m = local - pos * rt.half[axis];
-      // pos * theta^(-2m/D), D = 2 * half
-      double inv_freq = pow((double)a.theta, -(2.0 * m) / (2.0 * rt.half[axis]));
-      double ang = (double)pos * inv_freq;
-      double s, c;
-      sincos(ang, &s, &c);
-      tab[e] = make_float2((float)c, (float)s);
+      const int axis = (e >= rt.off[2]) ? 2 : (e >= rt.off[1]) ? 1 : 0;
+      const int local = e - rt.off[axis];
+      const int pos = local / rt.half[axis];
+      const int m = local - pos * rt.half[axis];
+      const int pair = m + (axis > 0 ? rt.half[0] : 0) + (axis > 1 ? rt.half[1] : 0);
+      double sn, cs;
+      sincos((double)pos * inv_freq[pair], &sn, &cs);  // angle pos * theta^(-2m/D) in fp64
+      tab[e] = make_float2((float)cs, (float)sn);
     }
     __syncthreads();
   }
@@ -109,12 +114,19 @@ __global__ void __launch_bounds__(kThreads) prologue_kernel(PrologueArgs a, Rope
       pw = rem - ph * a.W;
     }
 
+    // the next token's rows are loaded one iteration ahead, so that every
+    // thread keeps two 32-byte loads in flight
+    uint4 nq = make_uint4(0, 0, 0, 0), nk = make_uint4(0, 0, 0, 0);
+    if (active) {
+      nq = __ldcs(reinterpret_cast<const uint4*>(a.q + base + (size_t)n0 * row_stride));
+      nk = __ldcs(reinterpret_cast<const uint4*>(a.k + base + (size_t)n0 * row_stride));
+    }
     for (int n = n0; n < n1; ++n) {
       const size_t off = base + (size_t)n * row_stride;
-      uint4 vq = make_uint4(0, 0, 0, 0), vk = make_uint4(0, 0, 0, 0);
-      if (active) {
-        vq = __ldcs(reinterpret_cast<const uint4*>(a.q + off));
-        vk = __ldcs(reinterpret_cast<const uint4*>(a.k + off));
+      const uint4 vq = nq, vk = nk;
+      if (active && n + 1 < n1) {
+        nq = __ldcs(reinterpret_cast<const uint4*>(a.q + off + row_stride));
+        nk = __ldcs(reinterpret_cast<const uint4*>(a.k + off + row_stride));
       }
       float xq[8], xk[8];
       bf16x8_to_f32(vq, xq);
@@ -202,9 +214,14 @@ RopeTable make_table(const PrologueArgs& a) {
   return rt;
 }
 
-int grid_y_for(int nblk, int col_groups, int B, int sm_count) {
-  // about 6 resident 128-thread CTAs per SM
-  long want = (long)sm_count * 6 / ((long)col_groups * B);
+// Persistent grid: exactly as many CTAs as fit on the GPU at once (so there
+// is no partial second wave), split over column groups and batches.
+template <typename Kernel>
+int grid_y_for(Kernel k, size_t smem, int nblk, int col_groups, int B, int sm_count) {
+  int per_sm = 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, smem) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  long want = (long)sm_count * per_sm / ((long)col_groups * B);
   if (want < 1) want = 1;
   if (want > nblk) want = nblk;
   return (int)want;
@@ -223,18 +240,11 @@ int launch_prologue(const PrologueArgs& a, cudaStream_t stream) {
   const int col_groups = (a.H * kChunks + kThreads - 1) / kThreads;
   const RopeTable rt = make_table(a);
   const size_t smem = (size_t)rt.entries * sizeof(float2);
-  dim3 grid(col_groups, grid_y_for(a.nblk, col_groups, a.B, sms), a.B);
-  if (a.q_pool != nullptr) {
-    auto k = prologue_kernel<true, true>;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return SBATTN_ERR_CUDA;
-    k<<<grid, kThreads, smem, stream>>>(a, rt);
-  } else {
-    auto k = prologue_kernel<true, false>;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return SBATTN_ERR_CUDA;
-    k<<<grid, kThreads, smem, stream>>>(a, rt);
-  }
+  auto k = a.q_pool != nullptr ? prologue_kernel<true, true> : prologue_kernel<true, false>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return SBATTN_ERR_CUDA;
+  dim3 grid(col_groups, grid_y_for(k, smem, a.nblk, col_groups, a.B, sms), a.B);
+  k<<<grid, kThreads, smem, stream>>>(a, rt);
   return cudaGetLastError() == cudaSuccess ? SBATTN_OK : SBATTN_ERR_CUDA;
 }
 
@@ -243,9 +253,10 @@ int launch_pool(const PrologueArgs& a, cudaStream_t stream) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int col_groups = (a.H * kChunks + kThreads - 1) / kThreads;
-  dim3 grid(col_groups, grid_y_for(a.nblk, col_groups, a.B, sms), a.B);
+  auto k = prologue_kernel<false, true>;
+  dim3 grid(col_groups, grid_y_for(k, 0, a.nblk, col_groups, a.B, sms), a.B);
   RopeTable rt{};
-  prologue_kernel<false, true><<<grid, kThreads, 0, stream>>>(a, rt);
+  k<<<grid, kThreads, 0, stream>>>(a, rt);
   return cudaGetLastError() == cudaSuccess ? SBATTN_OK : SBATTN_ERR_CUDA;
 }
 

@@ -28,6 +28,8 @@ CASES = {
     "tiny": WORKLOADS["tiny"],
     "dense": WORKLOADS["dense"],
     "dense_s075": WORKLOADS["dense"].with_sparsity(0.75),
+    # K = 61: an odd number of tiles per item, ~14 items per CTA
+    "dense_odd": WORKLOADS["dense"].with_sparsity(0.76),
     "ragged": custom_workload("ragged", B=2, H=3, T=3, Hh=7, W=13, sparsity=0.6, seed=21),  # N = 273
     "odd_keep": custom_workload("odd_keep", B=1, H=4, T=2, Hh=16, W=30, sparsity=0.5, seed=22),  # nblk 15, K 8
     "one_block": custom_workload("one_block", B=1, H=2, T=1, Hh=5, W=7, sparsity=0.5, seed=23),  # N = 35
@@ -36,7 +38,7 @@ CASES = {
 
 # heads compared element by element (the kernels always run every head); the
 # dense check's fp64 attention is costly, so two of its eight heads are used
-HEADS = {"dense": (0, 5), "dense_s075": (1, 6)}
+HEADS = {"dense": (0, 5), "dense_s075": (1, 6), "dense_odd": (2, 7)}
 
 _ORACLE_ATTN = {}
 
