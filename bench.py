@@ -36,7 +36,7 @@ if ROOT not in sys.path:
 
 METRIC = "block-sparse attn ms/layer & eff. TFLOP/s (% bf16 peak); prologue GB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attention_traffic.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attention_traffic.txt")
 ATTN_SRC = os.path.join(ROOT, "block_sparse_attention_qk_b200", "csrc", "attention.cu")
 SWEEP = (0.5, 0.75, 0.8, 0.9)
 
@@ -109,10 +109,16 @@ def source_hash(path=ATTN_SRC) -> str:
 def recorded_traffic(workload: str, heads: int):
     """DRAM bytes per attention launch from the committed ncu summary, scaled
     to this workload; None if absent or if the kernel source has changed."""
+    rec = {}
     try:
         with open(TRAFFIC_FILE) as f:
-            rec = json.load(f)
-    except (OSError, ValueError):
+            for line in f:
+                key, sep, val = line.partition(":")
+                if sep and not line.startswith("#"):
+                    rec[key.strip()] = val.strip()
+    except OSError:
+        return None
+    if "dram_bytes_per_launch" not in rec or "heads" not in rec:
         return None
     if rec.get("source_sha256_16") != source_hash():
         return None
