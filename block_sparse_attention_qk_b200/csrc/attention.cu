@@ -12,35 +12,44 @@
 //
 // A key tile is two kept 64-token blocks, each fetched by TMA (two 64-channel
 // boxes per block, 128-byte swizzle) straight into the canonical operand
-// layout.  TMEM holds two S^T buffers (64 columns each) and the O^T
-// accumulator (64 columns); TMEM lane = key row for S, = channel for O.
+// layout.  TMEM holds a ring of four S^T tiles (64 columns each) and four
+// partial O^T accumulators; TMEM lane = key row for S, = channel for O.
 //
-// Tensor-core issue, measured on B200: a tcgen05.mma costs the issuing
-// thread about 146 cycles when it accumulates into the same TMEM tile as the
-// MMA before it, whatever its N, and about 73 cycles when the issue stream
-// rotates over eight accumulators.  An M=128, N=64, K=16 MMA has 32 cycles of
-// math; PV of a tile is therefore spread over four partial O^T accumulators
-// (K-step kk into partial kk mod 4; the epilogue sums them), and QK^T runs
-// into a ring of four S^T tiles.
+// Tensor-core issue, measured on B200: with N = 64 an MMA has only 32 cycles
+// of math, and the bound is how fast one thread can issue tcgen05.mma (about
+// 54 cycles apart in a tight loop, 120 with address arithmetic in between)
+// and the ~146-cycle latency of an MMA that accumulates into the tile the
+// previous one wrote.  Two warps therefore issue MMAs, each from a tight,
+// unrolled loop: one the QK^T chain of each tile into a ring of four S^T
+// tiles in TMEM, the other PV, spread over four partial O^T accumulators
+// (K-step kk into partial kk mod 4; the epilogue sums them), so that the two
+// streams interleave in the tensor pipe.  TMA streaming and MMAs on the same
+// SM do not slow each other down.
+//
+// Shared memory: Q (one stage), K and V (three stages each, so that a copy
+// has time to land while two tiles are in compute) and one P^T buffer
+// released in two key halves: the softmax threads of key rows 0-63 may write
+// the next P^T as soon as the first four PV K-steps are done, and the PV
+// issuer waits for the second half only before the last four.
 //
 // Two softmax work-groups of 128 threads split the 64 query columns of every
 // tile (32 each); a thread owns one TMEM lane, i.e. one KEY row across its 32
-// queries, and handles two tiles per step.  The per-query running maximum m
-// is seeded from the first step of the item (one cross-lane reduction per
-// item).  Later steps need no barrier: a thread that meets a logit more than
-// 2^8 above m raises a flag and records the excess per query (atomicMax); the
-// work-group reads the flag at the start of the next step, once every thread
-// has finished the previous one, and only then -- rarely -- raises m and
-// rescales O and the partial row sums.  The flagged step's p values stay
-// exact meanwhile: exp2 is only clamped beyond 2^100, which is reported as a
-// device error.  Each thread keeps 32 partial row sums, reduced once per item.
+// queries.  The per-query running maximum m is seeded from the first tile of
+// the item (one cross-lane reduction per item).  Later tiles need no barrier:
+// a thread that meets a logit more than 2^8 above m raises a flag and records
+// the excess per query (atomicMax); the work-group reads the flag at the start
+// of the next tile, once every softmax thread has stored its P^T of the
+// previous one, and only then -- rarely -- raises m and rescales O and the
+// partial row sums.  The flagged tile's p values stay exact meanwhile: exp2 is
+// only clamped beyond 2^100, which is reported as a device error.  Each thread
+// keeps 32 partial row sums, reduced once per item.
 //
 // Roles (384 threads, one CTA per SM, persistent over items):
 //   warp 0: TMA producer for Q and K tiles; also writes each tile's count of
 //           valid key rows into a small shared ring, so that the softmax
 //           warps never read the kept lists
-//   warp 1: TMA producer for V tiles           warp 2: TMEM allocator + MMA issuer
-//   warp 3: idle
+//   warp 1: TMA producer for V tiles
+//   warp 2: TMEM allocator + QK^T issuer       warp 3: PV issuer
 //   warps 4-7 and 8-11: softmax + epilogue work-groups for query columns
 //   0-31 and 32-63 (TMEM lane quarter = warp % 4)
 // Every mbarrier wait is bounded (2 s); on expiry the kernel records
@@ -63,15 +72,12 @@ constexpr int kInfoSlots = 16;        // per-tile valid-row counts, ring
 constexpr int kQBytes = 64 * 128 * 2;    // [2 channel halves][64 rows][128 B]
 constexpr int kKVBytes = 128 * 128 * 2;  // [2 channel halves][128 rows][128 B]
 constexpr int kPBytes = 128 * 64 * 2;    // [128 keys][64 queries] bf16
-// Shared-memory rings.  A V stage waits for the softmax's P before PV frees
-// it, so V gets the third stage; Q is reloaded once per item, covered by the
-// QK^T front running ahead.
-constexpr int kQStages = 1, kKStages = 2, kVStages = 3, kPStages = 2;
+constexpr int kQStages = 1, kKStages = 3, kVStages = 3;
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kQStages * kQBytes;
 constexpr int kOffV = kOffK + kKStages * kKVBytes;
 constexpr int kOffP = kOffV + kVStages * kKVBytes;
-constexpr int kOffMisc = kOffP + kPStages * kPBytes;
+constexpr int kOffMisc = kOffP + kPBytes;
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kExpClamp = 100.0f;         // p <= 2^100: sums stay finite
@@ -82,23 +88,23 @@ struct Misc {
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[kSBufs], s_empty[kSBufs];
-  uint64_t p_full[kPStages], p_empty[kPStages];
+  uint64_t p_full[2], p_empty[2];  // per key half (rows 0-63, 64-127) of the P^T buffer
   uint64_t o_full, o_empty;
   uint64_t info_full[kInfoSlots];
   uint64_t wg_bar[2];  // barrier of each softmax work-group (bounded wait)
-  uint64_t drain;
+  uint64_t drain[2];  // per MMA issuer, for the error path
   uint32_t info[kInfoSlots];  // valid key rows of a tile: low half | high half << 8
   uint32_t tmem_base;
   int abort;
   int flag[2][2];                 // per work-group, per step parity: a logit exceeded m by 2^8
   uint32_t raise_req[2][2][32];   // per work-group, per step parity: max excess per query (float bits)
-  float m2[64];         // running max per query, scaled to log2 units
+  alignas(16) float m2[64];  // running max per query, scaled to log2 units (read as float4)
   float alpha[64];      // rescale factors / final 1/l
-  float raise[64];      // increase of m in the current rescale
   float red[2][4][32];  // cross-warp reduction scratch per work-group
 };
 
-constexpr int kSmemBytes = kOffMisc + (int)sizeof(Misc) + 1024;  // + alignment slack
+static_assert(offsetof(Misc, m2) % 16 == 0, "m2 is read with 16-byte loads");
+constexpr int kSmemBytes = kOffMisc + (int)sizeof(Misc);  // base is 1024-byte aligned (checked)
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 64, 0, 0);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 64, 1, 1);
@@ -239,13 +245,16 @@ struct TileStream {
 __global__ void __launch_bounds__(kThreads, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, AttentionArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
   Misc* ms = reinterpret_cast<Misc*>(smem + kOffMisc);
   const uint32_t sbase = smem_addr(smem);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = a.B * a.H * a.nblk;
+  if ((sbase & 1023u) != 0u) {  // the 128-byte swizzle atoms need 1024-byte alignment
+    if (threadIdx.x == 0) record_error(a.status, SBATTN_ERR_DEVICE);
+    return;
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kQStages; ++s) {
@@ -260,8 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ms->v_full[s], 1);
       mbar_init(&ms->v_empty[s], 1);
     }
-    for (int s = 0; s < kPStages; ++s) {
-      mbar_init(&ms->p_full[s], kSoftmaxThreads);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&ms->p_full[s], kSoftmaxThreads / 2);
       mbar_init(&ms->p_empty[s], 1);
     }
     for (int s = 0; s < kSBufs; ++s) {
@@ -271,7 +280,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kInfoSlots; ++s) mbar_init(&ms->info_full[s], 1);
     mbar_init(&ms->wg_bar[0], 128);
     mbar_init(&ms->wg_bar[1], 128);
-    mbar_init(&ms->drain, 1);
+    mbar_init(&ms->drain[0], 1);
+    mbar_init(&ms->drain[1], 1);
     mbar_init(&ms->o_full, 1);
     mbar_init(&ms->o_empty, kSoftmaxThreads);
     ms->abort = 0;
@@ -373,93 +383,66 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ MMA issuer
-    // One thread walks the tile stream twice: the QK^T front (bounded by the
-    // S ring and the K ring) and the PV front (bounded by P and V); it issues
-    // a whole tile of whichever front is ready, polling both.
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ MMA issuers
+    // Warp 2 issues QK^T (bounded by the S ring and the K ring), warp 3 PV
+    // (bounded by P, V and the O accumulators).  With N = 64 every MMA has
+    // only 32 cycles of math, so the issuing thread's own instruction latency
+    // matters: the loops are unrolled over the K-steps and step precomputed
+    // descriptors by constants (+32 B inside the 128-byte atom = +2 in the
+    // descriptor's address field, which cannot carry for shared addresses).
+    const bool is_qk = warp == 2;
     bool ok = true;
     if (lane == 0) {
-      TileStream qk, pv;
-      qk.init(a, total);
-      pv.init(a, total);
-      uint32_t gq = 0, gp = 0;  // global tile counts of the two fronts
-      uint32_t inited = 0u;     // partial O accumulators started in the current item
-      int qsb[2], qks[2], qqb[2];
-      bool qlast[2];
-      // Wait for the inputs of the next QK^T tile and take it from the front.
-      auto qk_take = [&](int j) -> bool {
-        qsb[j] = gq % kSBufs;
-        qks[j] = gq % kKStages;
-        qqb[j] = qk.n % kQStages;
-        qlast[j] = qk.t == qk.it.ntiles - 1;
-        if (!mbar_wait(&ms->s_empty[qsb[j]], ((gq / kSBufs) & 1) ^ 1, abort_flag)) return false;
-        if (!mbar_wait(&ms->k_full[qks[j]], (gq / kKStages) & 1, abort_flag)) return false;
-        if (qk.t == 0 && !mbar_wait(&ms->q_full[qqb[j]], (qk.n / kQStages) & 1, abort_flag)) return false;
-        ++gq;
-        qk.advance(a, total);
-        return true;
-      };
-      auto qk_step = [&](int j, int kk) {
-        const uint32_t k_addr = sbase + kOffK + qks[j] * kKVBytes + (kk >> 2) * 16384 + (kk & 3) * 32;
-        const uint32_t q_addr = sbase + kOffQ + qqb[j] * kQBytes + (kk >> 2) * 8192 + (kk & 3) * 32;
-        umma_bf16(tmem + qsb[j] * 64, smem_desc(k_addr, 16, 1024, kSwizzle128B),
-                  smem_desc(q_addr, 16, 1024, kSwizzle128B), kIdescQK, kk > 0);
-      };
-      auto qk_commit = [&](int j) {
-        umma_commit(&ms->s_full[qsb[j]]);
-        umma_commit(&ms->k_empty[qks[j]]);
-        if (qlast[j]) umma_commit(&ms->q_empty[qqb[j]]);
-      };
-      uint64_t last = global_timer_ns();
-      while (pv.item < total) {
-        bool progressed = false;
-        // ---- QK^T front: a whole tile whenever its S slot and K are ready
-        // (the S ring bounds it to four tiles ahead of the softmax)
-        if (qk.item < total && mbar_test_wait(&ms->s_empty[gq % kSBufs], ((gq / kSBufs) & 1) ^ 1) &&
-            mbar_test_wait(&ms->k_full[gq % kKStages], (gq / kKStages) & 1) &&
-            (qk.t > 0 || mbar_test_wait(&ms->q_full[qk.n % kQStages], (qk.n / kQStages) & 1))) {
-          ok = qk_take(0);  // (its waits are already satisfied)
+      TileStream ts;
+      ts.init(a, total);
+      uint32_t gt = 0;  // global tile count of this front
+      while (ts.item < total) {
+        if (is_qk) {
+          const int sb = gt % kSBufs, ks = gt % kKStages, qb = ts.n % kQStages;
+          const bool last = ts.t == ts.it.ntiles - 1;
+          ok = mbar_wait(&ms->s_empty[sb], ((gt / kSBufs) & 1) ^ 1, abort_flag) &&
+               mbar_wait(&ms->k_full[ks], (gt / kKStages) & 1, abort_flag) &&
+               (ts.t > 0 || mbar_wait(&ms->q_full[qb], (ts.n / kQStages) & 1, abort_flag));
           if (!ok) break;
           tc_fence_after();
-          for (int kk = 0; kk < 8; ++kk) qk_step(0, kk);
-          qk_commit(0);
-          progressed = true;
-        }
-        // ---- PV front: a whole tile once its P and V are ready, its K-steps
-        // spread over the four partial O accumulators
-        const int ps = gp % kPStages, vs = gp % kVStages;
-        if (mbar_test_wait(&ms->p_full[ps], (gp / kPStages) & 1) &&
-            mbar_test_wait(&ms->v_full[vs], (gp / kVStages) & 1) &&
-            (pv.t > 0 || mbar_test_wait(&ms->o_empty, (pv.n & 1) ^ 1))) {
-          const bool pfirst = pv.t == 0, plast = pv.t == pv.it.ntiles - 1;
-          tc_fence_after();
-          if (pfirst) inited = 0u;  // the first MMA of an item into each partial starts it
-          const uint32_t v_addr = sbase + kOffV + vs * kKVBytes;
-          const uint32_t p_addr = sbase + kOffP + ps * kPBytes;
+          const uint64_t kd = smem_desc(sbase + kOffK + ks * kKVBytes, 16, 1024, kSwizzle128B);
+          const uint64_t qd = smem_desc(sbase + kOffQ + qb * kQBytes, 16, 1024, kSwizzle128B);
+          const uint32_t d = tmem + sb * 64;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const int part = kk & (kOParts - 1);
-            umma_bf16(tmem + kColO + part * 64, smem_desc(v_addr + kk * 2048, 16384, 1024, kSwizzle128B),
-                      smem_desc(p_addr + kk * 2048, 8192, 1024, kSwizzle128B), kIdescPV, (inited >> part) & 1u);
-            inited |= 1u << part;
-          }
-          umma_commit(&ms->p_empty[ps]);
-          umma_commit(&ms->v_empty[vs]);
-          if (plast) umma_commit(&ms->o_full);
-          ++gp;
-          pv.advance(a, total);
-          progressed = true;
-        }
-        if (progressed) {
-          last = global_timer_ns();
+          for (int kk = 0; kk < 8; ++kk)
+            umma_bf16(d, kd + (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2), qd + (uint64_t)((kk >> 2) * 512 + (kk & 3) * 2),
+                      kIdescQK, kk > 0);
+          umma_commit(&ms->s_full[sb]);
+          umma_commit(&ms->k_empty[ks]);
+          if (last) umma_commit(&ms->q_empty[qb]);
         } else {
-          if (*abort_flag || global_timer_ns() - last > kWaitLimitNs) {
-            ok = false;
-            break;
-          }
-          __nanosleep(20);
+          const int vs = gt % kVStages;
+          const bool first = ts.t == 0, last = ts.t == ts.it.ntiles - 1;
+          ok = mbar_wait(&ms->v_full[vs], (gt / kVStages) & 1, abort_flag) &&
+               mbar_wait(&ms->p_full[0], gt & 1, abort_flag) &&
+               (!first || mbar_wait(&ms->o_empty, (ts.n & 1) ^ 1, abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t vd = smem_desc(sbase + kOffV + vs * kKVBytes, 16384, 1024, kSwizzle128B);
+          const uint64_t pd = smem_desc(sbase + kOffP, 8192, 1024, kSwizzle128B);
+          // K-step kk accumulates into partial kk mod 4; the first tile of an
+          // item starts each partial
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tmem + kColO + kk * 64, vd + (uint64_t)(kk * 128), pd + (uint64_t)(kk * 128), kIdescPV, !first);
+          umma_commit(&ms->p_empty[0]);  // key rows 0-63 of P^T are free again
+          if (!(ok = mbar_wait(&ms->p_full[1], gt & 1, abort_flag))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 4; kk < 8; ++kk)
+            umma_bf16(tmem + kColO + (kk & 3) * 64, vd + (uint64_t)(kk * 128), pd + (uint64_t)(kk * 128), kIdescPV, 1u);
+          umma_commit(&ms->p_empty[1]);
+          umma_commit(&ms->v_empty[vs]);
+          if (last) umma_commit(&ms->o_full);
         }
+        ++gt;
+        ts.advance(a, total);
       }
     }
     ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -467,9 +450,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         *abort_flag = 1;
         record_error(a.status, SBATTN_ERR_TIMEOUT);
-        umma_commit(&ms->drain);  // completes once every issued MMA is done
+        uint64_t* drain = &ms->drain[is_qk ? 0 : 1];
+        umma_commit(drain);  // completes once every MMA this thread issued is done
         const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(&ms->drain, 0) && global_timer_ns() - t0 < 100000000ull) {
+        while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < 100000000ull) {
         }
       }
       __syncwarp();
@@ -506,15 +490,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int q = 0; q < kQCols; ++q) l[q] = 0.f;
 
-      for (int tA = 0; tA < it.ntiles; tA += 2) {
-        const bool hasB = tA + 1 < it.ntiles;
-        const uint32_t gA = gt + tA, gB = gA + 1;
-        const int par = (tA >> 1) & 1;  // step parity within the item
-        if (tA > 0) {
-          // ---- the previous step's flag: read once every thread of the
-          // work-group has arrived on the P_full of that step's last tile
-          const uint32_t gp_prev = gA - 1;
-          ok = warp_wait(&ms->p_full[gp_prev % kPStages], (gp_prev / kPStages) & 1, abort_flag);
+      for (int t = 0; t < it.ntiles; ++t) {
+        const uint32_t gx = gt + t;
+        const int par = t & 1;  // tile parity within the item
+        if (t > 0) {
+          // ---- the previous tile's flag: read once every softmax thread has
+          // stored its P^T of that tile
+          const uint32_t gprev = gx - 1;
+          ok = warp_wait(&ms->p_full[0], gprev & 1, abort_flag) && warp_wait(&ms->p_full[1], gprev & 1, abort_flag);
           if (!ok) break;
           if (flag[par ^ 1]) {
             // ---- rare path: raise m, rescale O and the partial sums ----
@@ -525,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!(ok = wg())) break;
             // every PV issued so far must be complete before O is touched
-            ok = warp_wait(&ms->p_empty[gp_prev % kPStages], (gp_prev / kPStages) & 1, abort_flag);
+            ok = warp_wait(&ms->p_empty[0], gprev & 1, abort_flag) && warp_wait(&ms->p_empty[1], gprev & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll 1
@@ -547,33 +530,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (r == 0) flag[par ^ 1] = 0;
           }
         }
-        // ---- S^T of the step's tiles: this work-group's 32 query columns
-        ok = warp_wait(&ms->s_full[gA % kSBufs], (gA / kSBufs) & 1, abort_flag);
-        if (ok && hasB) ok = warp_wait(&ms->s_full[gB % kSBufs], (gB / kSBufs) & 1, abort_flag);
+        // ---- S^T of the tile: this work-group's 32 query columns
+        ok = warp_wait(&ms->s_full[gx % kSBufs], (gx / kSBufs) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        float x[2 * kQCols];  // [0, 32): tile A, [32, 64): tile B
-        tmem_ld_32cols(lane_addr + (gA % kSBufs) * 64 + col0, *reinterpret_cast<uint32_t(*)[32]>(x));
-        if (hasB) tmem_ld_32cols(lane_addr + (gB % kSBufs) * 64 + col0, *reinterpret_cast<uint32_t(*)[32]>(x + kQCols));
+        float x[kQCols];
+        tmem_ld_32cols(lane_addr + (gx % kSBufs) * 64 + col0, *reinterpret_cast<uint32_t(*)[32]>(x));
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(&ms->s_empty[gA % kSBufs]);
-        if (hasB) mbar_arrive(&ms->s_empty[gB % kSBufs]);
-        // ---- which of my key rows are real keys (written by the K producer)
-        ok = warp_wait(&ms->info_full[gA % kInfoSlots], (gA / kInfoSlots) & 1, abort_flag);
-        if (ok && hasB) ok = warp_wait(&ms->info_full[gB % kInfoSlots], (gB / kInfoSlots) & 1, abort_flag);
+        mbar_arrive(&ms->s_empty[gx % kSBufs]);
+        // ---- is my key row a real key (count written by the K producer)
+        ok = warp_wait(&ms->info_full[gx % kInfoSlots], (gx / kInfoSlots) & 1, abort_flag);
         if (!ok) break;
-        const uint32_t infoA = ms->info[gA % kInfoSlots];
-        const uint32_t infoB = hasB ? ms->info[gB % kInfoSlots] : 0u;
-        const bool validA = (uint32_t)(r & 63) < ((infoA >> (8 * half)) & 0xFFu);
-        const bool validB = hasB && (uint32_t)(r & 63) < ((infoB >> (8 * half)) & 0xFFu);
+        const uint32_t info = ms->info[gx % kInfoSlots];
+        const bool valid = (uint32_t)(r & 63) < ((info >> (8 * half)) & 0xFFu);
 
-        if (tA == 0) {
-          // seed the running max from the first step
+        if (t == 0) {
+          // seed the running max from the first tile
           float v[kQCols];
 #pragma unroll
-          for (int q = 0; q < kQCols; ++q)
-            v[q] = fmaxf(validA ? x[q] * c : -INFINITY, validB ? x[q + kQCols] * c : -INFINITY);
+          for (int q = 0; q < kQCols; ++q) v[q] = valid ? x[q] * c : -INFINITY;
           const float mx = wg_reduce_cols<true>(v, red, quarter, lane, r, wg, ok);
           if (!ok) break;
           if (r < kQCols) m2[r] = (mx == -INFINITY) ? 0.f : mx;
@@ -588,51 +564,44 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int q = 4 * q4 + e;
-            x[q] = validA ? fmaf(x[q], c, -mm[e]) : -INFINITY;
-            x[q + kQCols] = validB ? fmaf(x[q + kQCols], c, -mm[e]) : -INFINITY;
-            lmax = fmaxf(lmax, fmaxf(x[q], x[q + kQCols]));
+            x[q] = valid ? fmaf(x[q], c, -mm[e]) : -INFINITY;
+            lmax = fmaxf(lmax, x[q]);
           }
         }
         if (lmax > kRescaleThreshold) {
-          // rare: ask the next step to raise m for these queries (logits are
+          // rare: ask the next tile to raise m for these queries (logits are
           // exact meanwhile up to 2^100 above m; beyond that they are clamped
           // and the call reports a device error)
 #pragma unroll
-          for (int q = 0; q < kQCols; ++q) {
-            const float ex = fmaxf(x[q], x[q + kQCols]);
-            if (ex > kRescaleThreshold) atomicMax(&raise_req[par][q], __float_as_uint(ex));
-          }
+          for (int q = 0; q < kQCols; ++q)
+            if (x[q] > kRescaleThreshold) atomicMax(&raise_req[par][q], __float_as_uint(x[q]));
           flag[par] = 1;
           if (lmax > kExpClamp) record_error(a.status, SBATTN_ERR_DEVICE);
         }
-        // ---- p = 2^x, partial row sums, bf16 P^T rows into shared memory:
+        // ---- p = 2^x, partial row sums, bf16 P^T row into shared memory:
         // row r of P^T holds 64 queries (128 B, 128-byte swizzle); this
         // work-group owns its 16-byte chunks 4g .. 4g + 3
+        uint32_t pk[kQCols / 2];
 #pragma unroll
-        for (int tile = 0; tile < 2; ++tile) {
-          if (tile == 1 && !hasB) break;
-          const uint32_t gx = gA + tile;
-          uint32_t pk[kQCols / 2];
-#pragma unroll
-          for (int q = 0; q < kQCols; q += 2) {
-            const float p0 = fast_exp2(fminf(x[tile * kQCols + q], kExpClamp));
-            const float p1 = fast_exp2(fminf(x[tile * kQCols + q + 1], kExpClamp));
-            l[q] += p0;
-            l[q + 1] += p1;
-            pk[q >> 1] = pack_bf16x2(p0, p1);
-          }
-          ok = warp_wait(&ms->p_empty[gx % kPStages], ((gx / kPStages) & 1) ^ 1, abort_flag);
-          if (!ok) break;
-          uint8_t* prow = smem + kOffP + (gx % kPStages) * kPBytes + r * 128;
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4)
-            *reinterpret_cast<uint4*>(prow + (((4 * g + c4) ^ (r & 7)) * 16)) =
-                make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
+        for (int q = 0; q < kQCols; q += 2) {
+          const float p0 = fast_exp2(fminf(x[q], kExpClamp));
+          const float p1 = fast_exp2(fminf(x[q + 1], kExpClamp));
+          pk[q >> 1] = pack_bf16x2(p0, p1);
+          // the row sums take the bf16 weights PV actually uses, so that O / l
+          // stays a convex combination of V rows even where no p is 1
+          l[q] += __uint_as_float(pk[q >> 1] << 16);
+          l[q + 1] += __uint_as_float(pk[q >> 1] & 0xFFFF0000u);
         }
+        // my half of the buffer is free once PV of the previous tile has read it
+        ok = warp_wait(&ms->p_empty[half], (gx & 1) ^ 1, abort_flag);
         if (!ok) break;
+        uint8_t* prow = smem + kOffP + r * 128;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4)
+          *reinterpret_cast<uint4*>(prow + (((4 * g + c4) ^ (r & 7)) * 16)) =
+              make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
         fence_proxy_async_smem();
-        mbar_arrive(&ms->p_full[gA % kPStages]);
-        if (hasB) mbar_arrive(&ms->p_full[gB % kPStages]);
+        mbar_arrive(&ms->p_full[half]);
       }
       if (!ok) break;
       gt += it.ntiles;
