@@ -72,14 +72,19 @@ constexpr int kInfoSlots = 16;        // per-tile valid-row counts, ring
 constexpr int kQBytes = 64 * 128 * 2;    // [2 channel halves][64 rows][128 B]
 constexpr int kKVBytes = 128 * 128 * 2;  // [2 channel halves][128 rows][128 B]
 constexpr int kPBytes = 128 * 64 * 2;    // [128 keys][64 queries] bf16
-constexpr int kQStages = 1, kKStages = 3, kVStages = 3;
+constexpr int kQStages = 1, kKStages = 3, kVStages = 2, kPStages = 2;
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kQStages * kQBytes;
 constexpr int kOffV = kOffK + kKStages * kKVBytes;
 constexpr int kOffP = kOffV + kVStages * kKVBytes;
-constexpr int kOffMisc = kOffP + kPBytes;
+constexpr int kOffMisc = kOffP + kPStages * kPBytes;
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// A flag raised at tile t is read at tile t + kFlagDelay: by then every
+// softmax thread has finished tile t (the P^T ring orders them), so all read
+// the same value without a barrier.  Slots are reused every kFlagSlots tiles.
+constexpr int kFlagDelay = 4;
+constexpr int kFlagSlots = 8;
 constexpr float kExpClamp = 100.0f;         // p <= 2^100: sums stay finite
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -88,7 +93,7 @@ struct Misc {
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[kSBufs], s_empty[kSBufs];
-  uint64_t p_full[2], p_empty[2];  // per key half (rows 0-63, 64-127) of the P^T buffer
+  uint64_t p_full[kPStages][2], p_empty[kPStages][2];  // per P^T buffer and key half (rows 0-63, 64-127)
   uint64_t o_full, o_empty;
   uint64_t info_full[kInfoSlots];
   uint64_t wg_bar[2];  // barrier of each softmax work-group (bounded wait)
@@ -96,8 +101,8 @@ struct Misc {
   uint32_t info[kInfoSlots];  // valid key rows of a tile: low half | high half << 8
   uint32_t tmem_base;
   int abort;
-  int flag[2][2];                 // per work-group, per step parity: a logit exceeded m by 2^8
-  uint32_t raise_req[2][2][32];   // per work-group, per step parity: max excess per query (float bits)
+  int flag[2][kFlagSlots];  // per work-group, per tile slot: a logit exceeded m by 2^8
+  uint32_t raise_req[2][32];  // per work-group: max excess per query (float bits) since the last rescale
   alignas(16) float m2[64];  // running max per query, scaled to log2 units (read as float4)
   float alpha[64];      // rescale factors / final 1/l
   float red[2][4][32];  // cross-warp reduction scratch per work-group
@@ -269,10 +274,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ms->v_full[s], 1);
       mbar_init(&ms->v_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&ms->p_full[s], kSoftmaxThreads / 2);
-      mbar_init(&ms->p_empty[s], 1);
-    }
+    for (int s = 0; s < kPStages; ++s)
+      for (int h = 0; h < 2; ++h) {
+        mbar_init(&ms->p_full[s][h], kSoftmaxThreads / 2);
+        mbar_init(&ms->p_empty[s][h], 1);
+      }
     for (int s = 0; s < kSBufs; ++s) {
       mbar_init(&ms->s_full[s], 1);
       mbar_init(&ms->s_empty[s], kSoftmaxThreads);
@@ -285,8 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&ms->o_full, 1);
     mbar_init(&ms->o_empty, kSoftmaxThreads);
     ms->abort = 0;
-    ms->flag[0][0] = ms->flag[0][1] = ms->flag[1][0] = ms->flag[1][1] = 0;
-    for (int e = 0; e < 2 * 2 * 32; ++e) (&ms->raise_req[0][0][0])[e] = 0u;
+    for (int e = 0; e < 2 * kFlagSlots; ++e) (&ms->flag[0][0])[e] = 0;
+    for (int e = 0; e < 2 * 32; ++e) (&ms->raise_req[0][0])[e] = 0u;
     fence_barrier_init();
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
@@ -417,27 +423,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(&ms->k_empty[ks]);
           if (last) umma_commit(&ms->q_empty[qb]);
         } else {
-          const int vs = gt % kVStages;
+          const int vs = gt % kVStages, pb = gt % kPStages;
+          const uint32_t pph = (gt / kPStages) & 1;
           const bool first = ts.t == 0, last = ts.t == ts.it.ntiles - 1;
           ok = mbar_wait(&ms->v_full[vs], (gt / kVStages) & 1, abort_flag) &&
-               mbar_wait(&ms->p_full[0], gt & 1, abort_flag) &&
+               mbar_wait(&ms->p_full[pb][0], pph, abort_flag) &&
                (!first || mbar_wait(&ms->o_empty, (ts.n & 1) ^ 1, abort_flag));
           if (!ok) break;
           tc_fence_after();
           const uint64_t vd = smem_desc(sbase + kOffV + vs * kKVBytes, 16384, 1024, kSwizzle128B);
-          const uint64_t pd = smem_desc(sbase + kOffP, 8192, 1024, kSwizzle128B);
+          const uint64_t pd = smem_desc(sbase + kOffP + pb * kPBytes, 8192, 1024, kSwizzle128B);
           // K-step kk accumulates into partial kk mod 4; the first tile of an
           // item starts each partial
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             umma_bf16(tmem + kColO + kk * 64, vd + (uint64_t)(kk * 128), pd + (uint64_t)(kk * 128), kIdescPV, !first);
-          umma_commit(&ms->p_empty[0]);  // key rows 0-63 of P^T are free again
-          if (!(ok = mbar_wait(&ms->p_full[1], gt & 1, abort_flag))) break;
+          umma_commit(&ms->p_empty[pb][0]);  // key rows 0-63 of this P^T buffer are free again
+          if (!(ok = mbar_wait(&ms->p_full[pb][1], pph, abort_flag))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 4; kk < 8; ++kk)
             umma_bf16(tmem + kColO + (kk & 3) * 64, vd + (uint64_t)(kk * 128), pd + (uint64_t)(kk * 128), kIdescPV, 1u);
-          umma_commit(&ms->p_empty[1]);
+          umma_commit(&ms->p_empty[pb][1]);
           umma_commit(&ms->v_empty[vs]);
           if (last) umma_commit(&ms->o_full);
         }
@@ -471,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* alpha = ms->alpha + col0;
     float(*red)[32] = ms->red[g];
     int* flag = ms->flag[g];
-    uint32_t(*raise_req)[32] = ms->raise_req[g];
+    uint32_t* raise_req = ms->raise_req[g];
     uint32_t gt = 0, on = 0;  // global tile index, item ordinal
     WgSync wg{&ms->wg_bar[g], abort_flag, 0};
     bool ok = true;
@@ -490,52 +497,51 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int q = 0; q < kQCols; ++q) l[q] = 0.f;
 
+      // S^T of tile t is loaded into x during tile t - 1 (the item's first
+      // one here), so that the TMEM load latency hides behind the P^T store
+      float x[kQCols];
+      ok = warp_wait(&ms->s_full[gt % kSBufs], (gt / kSBufs) & 1, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      tmem_ld_32cols(lane_addr + (gt % kSBufs) * 64 + col0, *reinterpret_cast<uint32_t(*)[32]>(x));
+
       for (int t = 0; t < it.ntiles; ++t) {
         const uint32_t gx = gt + t;
-        const int par = t & 1;  // tile parity within the item
-        if (t > 0) {
-          // ---- the previous tile's flag: read once every softmax thread has
-          // stored its P^T of that tile
-          const uint32_t gprev = gx - 1;
-          ok = warp_wait(&ms->p_full[0], gprev & 1, abort_flag) && warp_wait(&ms->p_full[1], gprev & 1, abort_flag);
-          if (!ok) break;
-          if (flag[par ^ 1]) {
-            // ---- rare path: raise m, rescale O and the partial sums ----
-            if (r < kQCols) {
-              const float up = __uint_as_float(raise_req[par ^ 1][r]);
-              alpha[r] = fast_exp2(-up);
-              m2[r] += up;
-            }
-            if (!(ok = wg())) break;
-            // every PV issued so far must be complete before O is touched
-            ok = warp_wait(&ms->p_empty[0], gprev & 1, abort_flag) && warp_wait(&ms->p_empty[1], gprev & 1, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-#pragma unroll 1
-            for (int part = 0; part < kOParts; ++part) {
-              uint32_t o[32];
-              const uint32_t oaddr = lane_addr + kColO + part * 64 + col0;
-              tmem_ld_32cols(oaddr, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int q = 0; q < kQCols; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha[q]);
-              tmem_st_32cols(oaddr, o);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-#pragma unroll
-            for (int q = 0; q < kQCols; ++q) l[q] *= alpha[q];
-            if (!(ok = wg())) break;  // everyone has read the request before it is cleared
-            if (r < kQCols) raise_req[par ^ 1][r] = 0u;
-            if (r == 0) flag[par ^ 1] = 0;
+        if (t >= kFlagDelay && flag[(t - kFlagDelay) & (kFlagSlots - 1)]) {
+          // ---- rare path: a logit of tile t - kFlagDelay (or later) exceeded m
+          // by 2^8; every thread of the work-group reads the same flag, as every
+          // thread finished that tile before any of them can be here.
+          if (!(ok = wg())) break;  // all threads are done with tile t - 1
+          if (r < kQCols) {
+            const float up = __uint_as_float(raise_req[r]);
+            alpha[r] = fast_exp2(-up);
+            m2[r] += up;
+            raise_req[r] = 0u;
           }
+          if (r < kFlagSlots) flag[r] = 0;
+          if (!(ok = wg())) break;
+          // every PV issued so far must be complete before O is touched
+          const uint32_t gp = gx - 1;
+          ok = warp_wait(&ms->p_empty[gp % 2][0], (gp / 2) & 1, abort_flag) &&
+               warp_wait(&ms->p_empty[gp % 2][1], (gp / 2) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int part = 0; part < kOParts; ++part) {
+            uint32_t o[32];
+            const uint32_t oaddr = lane_addr + kColO + part * 64 + col0;
+            tmem_ld_32cols(oaddr, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < kQCols; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha[q]);
+            tmem_st_32cols(oaddr, o);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+#pragma unroll
+          for (int q = 0; q < kQCols; ++q) l[q] *= alpha[q];
         }
-        // ---- S^T of the tile: this work-group's 32 query columns
-        ok = warp_wait(&ms->s_full[gx % kSBufs], (gx / kSBufs) & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        float x[kQCols];
-        tmem_ld_32cols(lane_addr + (gx % kSBufs) * 64 + col0, *reinterpret_cast<uint32_t(*)[32]>(x));
+        // ---- S^T of the tile (this work-group's 32 query columns) is in x
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&ms->s_empty[gx % kSBufs]);
@@ -569,18 +575,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (lmax > kRescaleThreshold) {
-          // rare: ask the next tile to raise m for these queries (logits are
+          // rare: ask a later tile to raise m for these queries (logits are
           // exact meanwhile up to 2^100 above m; beyond that they are clamped
           // and the call reports a device error)
 #pragma unroll
           for (int q = 0; q < kQCols; ++q)
-            if (x[q] > kRescaleThreshold) atomicMax(&raise_req[par][q], __float_as_uint(x[q]));
-          flag[par] = 1;
+            if (x[q] > kRescaleThreshold) atomicMax(&raise_req[q], __float_as_uint(x[q]));
+          flag[t & (kFlagSlots - 1)] = 1;
           if (lmax > kExpClamp) record_error(a.status, SBATTN_ERR_DEVICE);
         }
-        // ---- p = 2^x, partial row sums, bf16 P^T row into shared memory:
-        // row r of P^T holds 64 queries (128 B, 128-byte swizzle); this
-        // work-group owns its 16-byte chunks 4g .. 4g + 3
+        // ---- p = 2^x and partial row sums
         uint32_t pk[kQCols / 2];
 #pragma unroll
         for (int q = 0; q < kQCols; q += 2) {
@@ -592,16 +596,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           l[q] += __uint_as_float(pk[q >> 1] << 16);
           l[q + 1] += __uint_as_float(pk[q >> 1] & 0xFFFF0000u);
         }
-        // my half of the buffer is free once PV of the previous tile has read it
-        ok = warp_wait(&ms->p_empty[half], (gx & 1) ^ 1, abort_flag);
+        // ---- start loading the next tile's S^T
+        if (t + 1 < it.ntiles) {
+          const uint32_t gn = gx + 1;
+          ok = warp_wait(&ms->s_full[gn % kSBufs], (gn / kSBufs) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          tmem_ld_32cols(lane_addr + (gn % kSBufs) * 64 + col0, *reinterpret_cast<uint32_t(*)[32]>(x));
+        }
+        // ---- bf16 P^T row into shared memory once PV has released my half of
+        // the buffer: row r holds 64 queries (128 B, 128-byte swizzle); this
+        // work-group owns its 16-byte chunks 4g .. 4g + 3
+        const int pb = gx % 2;
+        ok = warp_wait(&ms->p_empty[pb][half], ((gx / 2) & 1) ^ 1, abort_flag);
         if (!ok) break;
-        uint8_t* prow = smem + kOffP + r * 128;
+        uint8_t* prow = smem + kOffP + pb * kPBytes + r * 128;
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4)
           *reinterpret_cast<uint4*>(prow + (((4 * g + c4) ^ (r & 7)) * 16)) =
               make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
         fence_proxy_async_smem();
-        mbar_arrive(&ms->p_full[half]);
+        mbar_arrive(&ms->p_full[pb][half]);
       }
       if (!ok) break;
       gt += it.ntiles;
@@ -611,8 +626,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       {
-        // a flag raised by the item's last step is moot: O is complete; clear it
-        // once every thread has finished that step (the o_full wait above)
+        // flags raised by the item's last tiles are moot: O is complete; clear
+        // them once every thread has finished the item (the o_full wait above)
         float v[kQCols];
 #pragma unroll
         for (int q = 0; q < kQCols; ++q) v[q] = l[q];
@@ -620,10 +635,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         if (r < kQCols) {
           alpha[r] = lsum > 0.f ? 1.0f / lsum : 0.f;
-          raise_req[0][r] = 0u;
-          raise_req[1][r] = 0u;
+          raise_req[r] = 0u;
         }
-        if (r == 0) flag[0] = flag[1] = 0;
+        if (r < kFlagSlots) flag[r] = 0;
         if (!(ok = wg())) break;
       }
       float acc[kQCols];
@@ -650,6 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (!ok) {
+      tmem_wait_ld();  // no TMEM load may be outstanding when the CTA frees TMEM
       if (r == 0) {
         *abort_flag = 1;
         record_error(a.status, SBATTN_ERR_TIMEOUT);
