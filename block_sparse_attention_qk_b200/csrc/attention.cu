@@ -34,15 +34,18 @@
 //
 // Two softmax work-groups of 128 threads split the 64 query columns of every
 // tile (32 each); a thread owns one TMEM lane, i.e. one KEY row across its 32
-// queries.  The per-query running maximum m is seeded from the first tile of
-// the item (one cross-lane reduction per item).  Later tiles need no barrier:
-// a thread that meets a logit more than 2^8 above m raises a flag and records
-// the excess per query (atomicMax); the work-group reads the flag at the start
-// of the next tile, once every softmax thread has stored its P^T of the
-// previous one, and only then -- rarely -- raises m and rescales O and the
-// partial row sums.  The flagged tile's p values stay exact meanwhile: exp2 is
-// only clamped beyond 2^100, which is reported as a device error.  Each thread
-// keeps 32 partial row sums, reduced once per item.
+// queries, and takes two tiles per step.  The per-query running maximum m is
+// seeded from the first step of the item (one cross-lane reduction per item).
+// Later steps need no barrier: a thread that meets a logit more than 2^8 above
+// m raises a flag and records the excess per query (atomicMax); the
+// work-group reads the flag three steps later, when the P^T ring guarantees
+// that every softmax thread has finished the flagged step, and only then --
+// rarely -- raises m (by the largest excess recorded so far) and rescales O
+// and the partial row sums.  The p values of the steps in between stay exact:
+// p up to 2^100 is fine in fp32 and bf16; a logit beyond that is reported as
+// a device error.  Each thread keeps 32 partial row sums (packed in pairs),
+// reduced once per item.  S^T of the next step is loaded from TMEM while the
+// current P^T is stored.
 //
 // Roles (384 threads, one CTA per SM, persistent over items):
 //   warp 0: TMA producer for Q and K tiles; also writes each tile's count of
@@ -80,12 +83,13 @@ constexpr int kOffP = kOffV + kVStages * kKVBytes;
 constexpr int kOffMisc = kOffP + kPStages * kPBytes;
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// A flag raised at tile t is read at tile t + kFlagDelay: by then every
-// softmax thread has finished tile t (the P^T ring orders them), so all read
-// the same value without a barrier.  Slots are reused every kFlagSlots tiles.
-constexpr int kFlagDelay = 4;
+// A flag raised in softmax step s (two tiles) is read in step s + kFlagDelay:
+// by then every softmax thread has finished step s (the P^T ring orders
+// them), so all read the same value without a barrier.  Slots are reused
+// every kFlagSlots steps.
+constexpr int kFlagDelay = 3;
 constexpr int kFlagSlots = 8;
-constexpr float kExpClamp = 100.0f;         // p <= 2^100: sums stay finite
+constexpr float kExpLimit = 100.0f;  // p > 2^100 is reported: sums might overflow
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Misc {
@@ -101,14 +105,14 @@ struct Misc {
   uint32_t info[kInfoSlots];  // valid key rows of a tile: low half | high half << 8
   uint32_t tmem_base;
   int abort;
-  int flag[2][kFlagSlots];  // per work-group, per tile slot: a logit exceeded m by 2^8
+  int flag[2][kFlagSlots];  // per work-group, per softmax-step slot: a logit exceeded m by 2^8
   uint32_t raise_req[2][32];  // per work-group: max excess per query (float bits) since the last rescale
-  alignas(16) float m2[64];  // running max per query, scaled to log2 units (read as float4)
+  alignas(16) float negm2[64];  // minus the running max per query, in log2 units (read as float4)
   float alpha[64];      // rescale factors / final 1/l
   float red[2][4][32];  // cross-warp reduction scratch per work-group
 };
 
-static_assert(offsetof(Misc, m2) % 16 == 0, "m2 is read with 16-byte loads");
+static_assert(offsetof(Misc, negm2) % 16 == 0, "negm2 is read with 16-byte loads");
 constexpr int kSmemBytes = kOffMisc + (int)sizeof(Misc);  // base is 1024-byte aligned (checked)
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 64, 0, 0);
@@ -474,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int col0 = kQCols * g;
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     const float c = a.scale * kLog2e;
-    float* m2 = ms->m2 + col0;
+    float* negm2 = ms->negm2 + col0;
     float* alpha = ms->alpha + col0;
     float(*red)[32] = ms->red[g];
     int* flag = ms->flag[g];
@@ -493,35 +497,48 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (q < qrows) obase[(size_t)q * row_stride] = 0;
         continue;
       }
-      float l[kQCols];
+      uint64_t l2[kQCols / 2];  // partial row sums, packed pairs of queries
 #pragma unroll
-      for (int q = 0; q < kQCols; ++q) l[q] = 0.f;
+      for (int q = 0; q < kQCols / 2; ++q) l2[q] = 0ull;
 
-      // S^T of tile t is loaded into x during tile t - 1 (the item's first
-      // one here), so that the TMEM load latency hides behind the P^T store
-      float x[kQCols];
-      ok = warp_wait(&ms->s_full[gt % kSBufs], (gt / kSBufs) & 1, abort_flag);
-      if (!ok) break;
-      tc_fence_after();
-      tmem_ld_32cols(lane_addr + (gt % kSBufs) * 64 + col0, *reinterpret_cast<uint32_t(*)[32]>(x));
+      // The softmax takes the item's tiles two at a time (a step), so that its
+      // fixed costs per wait are shared by 64 logits per thread.  S^T of a
+      // step's tiles is loaded into x during the previous step (the item's
+      // first step here), hiding the TMEM load latency behind the P^T stores.
+      // Barriers signalled in tile order by one thread (S^T full, info, P^T
+      // empty) are waited on for the later tile of a step only.
+      float x[2 * kQCols];  // [0, 32): tile A, [32, 64): tile B
+      {
+        const bool hasB = it.ntiles > 1;
+        const uint32_t gl = hasB ? gt + 1 : gt;
+        ok = warp_wait(&ms->s_full[gl % kSBufs], (gl / kSBufs) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        tmem_ld_32cols(lane_addr + (gt % kSBufs) * 64 + col0, *reinterpret_cast<uint32_t(*)[32]>(x));
+        if (hasB)
+          tmem_ld_32cols(lane_addr + ((gt + 1) % kSBufs) * 64 + col0, *reinterpret_cast<uint32_t(*)[32]>(x + kQCols));
+      }
 
-      for (int t = 0; t < it.ntiles; ++t) {
-        const uint32_t gx = gt + t;
-        if (t >= kFlagDelay && flag[(t - kFlagDelay) & (kFlagSlots - 1)]) {
-          // ---- rare path: a logit of tile t - kFlagDelay (or later) exceeded m
+      for (int tA = 0; tA < it.ntiles; tA += 2) {
+        const bool hasB = tA + 1 < it.ntiles;
+        const uint32_t gA = gt + tA, gB = gA + 1;
+        const uint32_t gl = hasB ? gB : gA;  // the step's last tile
+        const int step = tA >> 1;
+        if (step >= kFlagDelay && flag[(step - kFlagDelay) & (kFlagSlots - 1)]) {
+          // ---- rare path: a logit of step - kFlagDelay (or later) exceeded m
           // by 2^8; every thread of the work-group reads the same flag, as every
-          // thread finished that tile before any of them can be here.
-          if (!(ok = wg())) break;  // all threads are done with tile t - 1
+          // thread finished that step before any of them can be here.
+          if (!(ok = wg())) break;  // all threads are done with the previous step
           if (r < kQCols) {
             const float up = __uint_as_float(raise_req[r]);
             alpha[r] = fast_exp2(-up);
-            m2[r] += up;
+            negm2[r] -= up;
             raise_req[r] = 0u;
           }
           if (r < kFlagSlots) flag[r] = 0;
           if (!(ok = wg())) break;
           // every PV issued so far must be complete before O is touched
-          const uint32_t gp = gx - 1;
+          const uint32_t gp = gA - 1;
           ok = warp_wait(&ms->p_empty[gp % 2][0], (gp / 2) & 1, abort_flag) &&
                warp_wait(&ms->p_empty[gp % 2][1], (gp / 2) & 1, abort_flag);
           if (!ok) break;
@@ -539,84 +556,119 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_st();
           tc_fence_before();
 #pragma unroll
-          for (int q = 0; q < kQCols; ++q) l[q] *= alpha[q];
+          for (int q = 0; q < kQCols; q += 2) l2[q >> 1] = f2_mul(l2[q >> 1], f2_pack(alpha[q], alpha[q + 1]));
         }
-        // ---- S^T of the tile (this work-group's 32 query columns) is in x
+        // ---- S^T of the step's tiles (this work-group's 32 query columns) is in x
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(&ms->s_empty[gx % kSBufs]);
-        // ---- is my key row a real key (count written by the K producer)
-        ok = warp_wait(&ms->info_full[gx % kInfoSlots], (gx / kInfoSlots) & 1, abort_flag);
+        mbar_arrive(&ms->s_empty[gA % kSBufs]);
+        if (hasB) mbar_arrive(&ms->s_empty[gB % kSBufs]);
+        // ---- are my key rows real keys (counts written by the K producer)
+        ok = warp_wait(&ms->info_full[gl % kInfoSlots], (gl / kInfoSlots) & 1, abort_flag);
         if (!ok) break;
-        const uint32_t info = ms->info[gx % kInfoSlots];
-        const bool valid = (uint32_t)(r & 63) < ((info >> (8 * half)) & 0xFFu);
+        const uint32_t infoA = ms->info[gA % kInfoSlots];
+        const uint32_t infoB = hasB ? ms->info[gB % kInfoSlots] : 0u;
+        const bool validA = (uint32_t)(r & 63) < ((infoA >> (8 * half)) & 0xFFu);
+        const bool validB = (uint32_t)(r & 63) < ((infoB >> (8 * half)) & 0xFFu);
 
-        if (t == 0) {
-          // seed the running max from the first tile
+        if (tA == 0) {
+          // seed the running max from the first step
           float v[kQCols];
 #pragma unroll
-          for (int q = 0; q < kQCols; ++q) v[q] = valid ? x[q] * c : -INFINITY;
+          for (int q = 0; q < kQCols; ++q)
+            v[q] = fmaxf(validA ? x[q] * c : -INFINITY, validB ? x[q + kQCols] * c : -INFINITY);
           const float mx = wg_reduce_cols<true>(v, red, quarter, lane, r, wg, ok);
           if (!ok) break;
-          if (r < kQCols) m2[r] = (mx == -INFINITY) ? 0.f : mx;
+          if (r < kQCols) negm2[r] = (mx == -INFINITY) ? 0.f : -mx;
           if (!(ok = wg())) break;
         }
-        // ---- x <- s * c - m2 (log2 domain); rows outside the kept set -> -inf
+        // ---- x <- s * c - m (log2 domain), two lanes per instruction; rows
+        // outside the kept set -> -inf
         float lmax = -INFINITY;
+        {
+          const uint64_t c2 = f2_pack(c, c);
 #pragma unroll
-        for (int q4 = 0; q4 < kQCols / 4; ++q4) {
-          const float4 m4 = reinterpret_cast<const float4*>(m2)[q4];
-          const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+          for (int q4 = 0; q4 < kQCols / 4; ++q4) {
+            const float4 m4 = reinterpret_cast<const float4*>(negm2)[q4];
+            const uint64_t mlo = f2_pack(m4.x, m4.y), mhi = f2_pack(m4.z, m4.w);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int q = 4 * q4 + e;
-            x[q] = valid ? fmaf(x[q], c, -mm[e]) : -INFINITY;
-            lmax = fmaxf(lmax, x[q]);
+            for (int tile = 0; tile < 2; ++tile) {
+              const int q = tile * kQCols + 4 * q4;
+              const uint64_t a0 = f2_fma(f2_pack(x[q], x[q + 1]), c2, mlo);
+              const uint64_t a1 = f2_fma(f2_pack(x[q + 2], x[q + 3]), c2, mhi);
+              f2_unpack(a0, x[q], x[q + 1]);
+              f2_unpack(a1, x[q + 2], x[q + 3]);
+            }
           }
+          if (!validA) {
+#pragma unroll
+            for (int q = 0; q < kQCols; ++q) x[q] = -INFINITY;
+          }
+          if (!validB) {
+#pragma unroll
+            for (int q = 0; q < kQCols; ++q) x[kQCols + q] = -INFINITY;
+          }
+#pragma unroll
+          for (int q = 0; q < kQCols; q += 2)
+            lmax = fmax3(lmax, fmaxf(x[q], x[q + 1]), fmaxf(x[kQCols + q], x[kQCols + q + 1]));
         }
         if (lmax > kRescaleThreshold) {
-          // rare: ask a later tile to raise m for these queries (logits are
-          // exact meanwhile up to 2^100 above m; beyond that they are clamped
-          // and the call reports a device error)
+          // rare: ask a later step to raise m for these queries (logits are
+          // exact meanwhile up to 2^100 above m; beyond that the call reports
+          // a device error)
 #pragma unroll
-          for (int q = 0; q < kQCols; ++q)
-            if (x[q] > kRescaleThreshold) atomicMax(&raise_req[q], __float_as_uint(x[q]));
-          flag[t & (kFlagSlots - 1)] = 1;
-          if (lmax > kExpClamp) record_error(a.status, SBATTN_ERR_DEVICE);
+          for (int q = 0; q < kQCols; ++q) {
+            const float ex = fmaxf(x[q], x[kQCols + q]);
+            if (ex > kRescaleThreshold) atomicMax(&raise_req[q], __float_as_uint(ex));
+          }
+          flag[step & (kFlagSlots - 1)] = 1;
+          if (lmax > kExpLimit) record_error(a.status, SBATTN_ERR_DEVICE);
         }
-        // ---- p = 2^x and partial row sums
-        uint32_t pk[kQCols / 2];
+        // ---- p = 2^x and partial row sums (a row outside the kept set has
+        // x = -inf and p = 0); the row sums take the bf16 weights PV actually
+        // uses, so that O / l stays a convex combination of V rows even where
+        // no p is 1
+        uint32_t pk[2][kQCols / 2];
 #pragma unroll
-        for (int q = 0; q < kQCols; q += 2) {
-          const float p0 = fast_exp2(fminf(x[q], kExpClamp));
-          const float p1 = fast_exp2(fminf(x[q + 1], kExpClamp));
-          pk[q >> 1] = pack_bf16x2(p0, p1);
-          // the row sums take the bf16 weights PV actually uses, so that O / l
-          // stays a convex combination of V rows even where no p is 1
-          l[q] += __uint_as_float(pk[q >> 1] << 16);
-          l[q + 1] += __uint_as_float(pk[q >> 1] & 0xFFFF0000u);
+        for (int tile = 0; tile < 2; ++tile) {
+#pragma unroll
+          for (int q = 0; q < kQCols; q += 2) {
+            const int i = tile * kQCols + q;
+            pk[tile][q >> 1] = pack_bf16x2(fast_exp2(x[i]), fast_exp2(x[i + 1]));
+            l2[q >> 1] = f2_add(l2[q >> 1], f2_pack(__uint_as_float(pk[tile][q >> 1] << 16),
+                                                    __uint_as_float(pk[tile][q >> 1] & 0xFFFF0000u)));
+          }
         }
-        // ---- start loading the next tile's S^T
-        if (t + 1 < it.ntiles) {
-          const uint32_t gn = gx + 1;
-          ok = warp_wait(&ms->s_full[gn % kSBufs], (gn / kSBufs) & 1, abort_flag);
+        // ---- start loading the next step's S^T
+        if (tA + 2 < it.ntiles) {
+          const bool nB = tA + 3 < it.ntiles;
+          const uint32_t gn = gA + 2, gnl = nB ? gn + 1 : gn;
+          ok = warp_wait(&ms->s_full[gnl % kSBufs], (gnl / kSBufs) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
           tmem_ld_32cols(lane_addr + (gn % kSBufs) * 64 + col0, *reinterpret_cast<uint32_t(*)[32]>(x));
+          if (nB)
+            tmem_ld_32cols(lane_addr + ((gn + 1) % kSBufs) * 64 + col0, *reinterpret_cast<uint32_t(*)[32]>(x + kQCols));
         }
-        // ---- bf16 P^T row into shared memory once PV has released my half of
-        // the buffer: row r holds 64 queries (128 B, 128-byte swizzle); this
-        // work-group owns its 16-byte chunks 4g .. 4g + 3
-        const int pb = gx % 2;
-        ok = warp_wait(&ms->p_empty[pb][half], ((gx / 2) & 1) ^ 1, abort_flag);
-        if (!ok) break;
-        uint8_t* prow = smem + kOffP + pb * kPBytes + r * 128;
+        // ---- bf16 P^T rows into shared memory once PV has released my half
+        // of each buffer: row r holds 64 queries (128 B, 128-byte swizzle);
+        // this work-group owns its 16-byte chunks 4g .. 4g + 3
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4)
-          *reinterpret_cast<uint4*>(prow + (((4 * g + c4) ^ (r & 7)) * 16)) =
-              make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
-        fence_proxy_async_smem();
-        mbar_arrive(&ms->p_full[pb][half]);
+        for (int tile = 0; tile < 2; ++tile) {
+          if (tile == 1 && !hasB) break;
+          const uint32_t gx = gA + tile;
+          const int pb = gx % 2;
+          ok = warp_wait(&ms->p_empty[pb][half], ((gx / 2) & 1) ^ 1, abort_flag);
+          if (!ok) break;
+          uint8_t* prow = smem + kOffP + pb * kPBytes + r * 128;
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4)
+            *reinterpret_cast<uint4*>(prow + (((4 * g + c4) ^ (r & 7)) * 16)) =
+                make_uint4(pk[tile][4 * c4], pk[tile][4 * c4 + 1], pk[tile][4 * c4 + 2], pk[tile][4 * c4 + 3]);
+          fence_proxy_async_smem();
+          mbar_arrive(&ms->p_full[pb][half]);
+        }
+        if (!ok) break;
       }
       if (!ok) break;
       gt += it.ntiles;
@@ -630,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // them once every thread has finished the item (the o_full wait above)
         float v[kQCols];
 #pragma unroll
-        for (int q = 0; q < kQCols; ++q) v[q] = l[q];
+        for (int q = 0; q < kQCols; q += 2) f2_unpack(l2[q >> 1], v[q], v[q + 1]);
         const float lsum = wg_reduce_cols<false>(v, red, quarter, lane, r, wg, ok);
         if (!ok) break;
         if (r < kQCols) {
