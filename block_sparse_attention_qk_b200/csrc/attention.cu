@@ -665,10 +665,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c4 = 0; c4 < 4; ++c4)
             *reinterpret_cast<uint4*>(prow + (((4 * g + c4) ^ (r & 7)) * 16)) =
                 make_uint4(pk[tile][4 * c4], pk[tile][4 * c4 + 1], pk[tile][4 * c4 + 2], pk[tile][4 * c4 + 3]);
-          fence_proxy_async_smem();
-          mbar_arrive(&ms->p_full[pb][half]);
         }
         if (!ok) break;
+        // one proxy fence per step: it is cheap alone, but costly while the
+        // SM's async proxy is busy with copies and MMAs
+        fence_proxy_async_smem();
+        mbar_arrive(&ms->p_full[gA % 2][half]);
+        if (hasB) mbar_arrive(&ms->p_full[gB % 2][half]);
       }
       if (!ok) break;
       gt += it.ntiles;
