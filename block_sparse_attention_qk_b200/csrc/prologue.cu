@@ -114,19 +114,26 @@ __global__ void __launch_bounds__(kThreads) prologue_kernel(PrologueArgs a, Rope
       pw = rem - ph * a.W;
     }
 
-    // the next token's rows are loaded one iteration ahead, so that every
-    // thread keeps two 32-byte loads in flight
+    // the rows of the next two tokens are loaded ahead, so that every thread
+    // keeps four 16-byte loads in flight
     uint4 nq = make_uint4(0, 0, 0, 0), nk = make_uint4(0, 0, 0, 0);
+    uint4 mq = make_uint4(0, 0, 0, 0), mk = make_uint4(0, 0, 0, 0);
     if (active) {
       nq = __ldcs(reinterpret_cast<const uint4*>(a.q + base + (size_t)n0 * row_stride));
       nk = __ldcs(reinterpret_cast<const uint4*>(a.k + base + (size_t)n0 * row_stride));
+      if (n0 + 1 < n1) {
+        mq = __ldcs(reinterpret_cast<const uint4*>(a.q + base + (size_t)(n0 + 1) * row_stride));
+        mk = __ldcs(reinterpret_cast<const uint4*>(a.k + base + (size_t)(n0 + 1) * row_stride));
+      }
     }
     for (int n = n0; n < n1; ++n) {
       const size_t off = base + (size_t)n * row_stride;
       const uint4 vq = nq, vk = nk;
-      if (active && n + 1 < n1) {
-        nq = __ldcs(reinterpret_cast<const uint4*>(a.q + off + row_stride));
-        nk = __ldcs(reinterpret_cast<const uint4*>(a.k + off + row_stride));
+      nq = mq;
+      nk = mk;
+      if (active && n + 2 < n1) {
+        mq = __ldcs(reinterpret_cast<const uint4*>(a.q + off + 2 * row_stride));
+        mk = __ldcs(reinterpret_cast<const uint4*>(a.k + off + 2 * row_stride));
       }
       float xq[8], xk[8];
       bf16x8_to_f32(vq, xq);
