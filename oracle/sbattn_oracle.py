@@ -314,3 +314,48 @@ def dense_attention(q, k, v, scale=None) -> np.ndarray:
         scale = 1.0 / math.sqrt(d)
     s = np.einsum("bnhd,bmhd->bhnm", q, k) * scale
     return np.einsum("bhnm,bmhd->bnhd", softmax(s, axis=-1), v)
+
+
+# ----------------------------------------------------------------------------
+# the fused elementwise steps either side of attention in the DiT block
+# ([p3] "先把近两倍的免费收益拿走": the lossless gain includes fused AdaLN and
+# SwiGLU kernels).  The page names them only; the readings below are the
+# standard DiT definitions:
+#
+# * AdaLN: LayerNorm of each token's hidden vector without a learned affine
+#   (mean and biased variance over the C channels, eps inside the square
+#   root), then modulated by the per-sample conditioning vectors shift and
+#   scale: y = x_hat * (1 + scale) + shift;
+# * SwiGLU: the gated activation between the MLP's two projections,
+#   out = silu(gate) * up with silu(a) = a / (1 + exp(-a)), gate and up being
+#   the two halves of the first projection's output.
+
+
+def layer_norm(x: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """LayerNorm over the last axis without affine parameters:
+    (x - mean) / sqrt(var + eps) with the biased (1/C) variance."""
+    x = np.asarray(x, dtype=np.float64)
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps)
+
+
+def adaln_modulate(x: np.ndarray, shift: np.ndarray, scale: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """AdaLN of x [B, N, C] with per-sample shift, scale [B, C]:
+    layer_norm(x) * (1 + scale) + shift, float64."""
+    shift = np.asarray(shift, dtype=np.float64)[:, None, :]
+    scale = np.asarray(scale, dtype=np.float64)[:, None, :]
+    return layer_norm(x, eps) * (1.0 + scale) + shift
+
+
+def silu(a: np.ndarray) -> np.ndarray:
+    """a * sigmoid(a) = a / (1 + exp(-a)) in float64 (exp(-a) may overflow to
+    inf for very negative a, giving the correct limit -0)."""
+    a = np.asarray(a, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return a / (1.0 + np.exp(-a))
+
+
+def swiglu(gate: np.ndarray, up: np.ndarray) -> np.ndarray:
+    """SwiGLU gating: silu(gate) * up, elementwise, float64."""
+    return silu(gate) * np.asarray(up, dtype=np.float64)

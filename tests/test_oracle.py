@@ -366,3 +366,72 @@ def test_explicit_scale_matches_default():
     np.testing.assert_array_equal(a, b)
     c = orc.block_sparse_attention(q, k, v, idx, cnt, scale=0.5)
     assert not np.allclose(a, c)
+
+
+# ---------------------------------------------------------------- AdaLN / SwiGLU
+
+def test_layer_norm_hand_example():
+    # x = (1, 2, 3, 4): mean 5/2, biased variance 5/4, eps 0
+    y = orc.layer_norm(np.array([1.0, 2.0, 3.0, 4.0]), eps=0.0)
+    s = math.sqrt(1.25)
+    np.testing.assert_allclose(y, [-1.5 / s, -0.5 / s, 0.5 / s, 1.5 / s], rtol=0, atol=1e-15)
+
+
+def test_layer_norm_moments_closed_form():
+    # rows of y have mean 0 and variance var / (var + eps) exactly: catches a
+    # dropped mean, an unbiased variance or eps outside the square root
+    rng = np.random.default_rng(11)
+    x = rng.normal(2.0, 0.01, size=(3, 5, 64))
+    eps = 1e-4
+    y = orc.layer_norm(x, eps)
+    var = x.var(axis=-1)
+    np.testing.assert_allclose(y.mean(axis=-1), 0.0, atol=1e-12)
+    np.testing.assert_allclose((y ** 2).mean(axis=-1), var / (var + eps), rtol=1e-12)
+
+
+def test_layer_norm_is_affine_invariant():
+    rng = np.random.default_rng(12)
+    x = rng.normal(size=(2, 3, 48))
+    np.testing.assert_allclose(orc.layer_norm(3.5 * x - 7.0, 0.0), orc.layer_norm(x, 0.0), atol=1e-12)
+
+
+def test_adaln_modulation_special_cases():
+    rng = np.random.default_rng(13)
+    x = rng.normal(size=(2, 4, 32))
+    shift = rng.normal(size=(2, 32))
+    zero = np.zeros((2, 32))
+    # scale = shift = 0 -> plain LayerNorm; scale = -1 -> shift regardless of x
+    np.testing.assert_allclose(orc.adaln_modulate(x, zero, zero), orc.layer_norm(x), atol=1e-15)
+    np.testing.assert_allclose(orc.adaln_modulate(x, shift, -np.ones((2, 32))),
+                               np.broadcast_to(shift[:, None, :], x.shape), atol=1e-15)
+    # constant rows normalise to 0 -> shift
+    c = np.full((2, 4, 32), 3.25)
+    np.testing.assert_allclose(orc.adaln_modulate(c, shift, rng.normal(size=(2, 32))),
+                               np.broadcast_to(shift[:, None, :], c.shape), atol=1e-15)
+    # (1 + scale), per sample: doubling the normalised row needs scale = 1
+    np.testing.assert_allclose(orc.adaln_modulate(x, zero, np.ones((2, 32))), 2 * orc.layer_norm(x), atol=1e-14)
+    # sample b uses its own vectors
+    s2 = np.stack([np.zeros(32), np.full(32, 5.0)])
+    y = orc.adaln_modulate(x, s2, zero)
+    np.testing.assert_allclose(y[1] - y[0], 5.0 + orc.layer_norm(x)[1] - orc.layer_norm(x)[0], atol=1e-13)
+
+
+def test_silu_values_and_identity():
+    assert orc.silu(np.array(0.0)) == 0.0
+    np.testing.assert_allclose(orc.silu(np.array([1.0, -1.0])), [1 / (1 + math.exp(-1)), -1 / (1 + math.e)], rtol=1e-15)
+    a = np.linspace(-30, 30, 121)
+    # silu(a) - silu(-a) = a (a * (sigmoid(a) + sigmoid(-a)))
+    np.testing.assert_allclose(orc.silu(a) - orc.silu(-a), a, atol=1e-13)
+    big = orc.silu(np.array([-1000.0, 1000.0]))
+    assert big[0] == 0.0 and big[1] == 1000.0
+    # silu against torch's SiLU on the same fp64 values
+    np.testing.assert_allclose(orc.silu(a), torch.nn.functional.silu(torch.from_numpy(a)).numpy(), rtol=1e-14, atol=1e-300)
+
+
+def test_swiglu_gates_up():
+    rng = np.random.default_rng(14)
+    g = rng.normal(size=(5, 16))
+    u = rng.normal(size=(5, 16))
+    np.testing.assert_allclose(orc.swiglu(g, np.ones_like(g)), orc.silu(g), atol=0)
+    np.testing.assert_allclose(orc.swiglu(g, 2 * u), 2 * orc.swiglu(g, u), rtol=1e-15)
+    assert not np.allclose(orc.swiglu(g, u), orc.swiglu(u, g))  # gate and up are not interchangeable
