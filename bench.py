@@ -44,6 +44,7 @@ SWEEP = (0.5, 0.75, 0.8, 0.9)
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--no-dit", action="store_true", help="skip the AdaLN / SwiGLU measurement")
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
@@ -271,6 +272,51 @@ def config_of(wl, K, n_gpus):
             "l2_policy": "inputs (3 x B*N*H*d bf16) larger than the 126 MB L2; no flush"}
 
 
+def measure_dit_ops(sb, x, wl, dev, peaks, iters=5):
+    """The fused elementwise steps either side of attention, at this layer's
+    size: AdaLN on the hidden states [B, N, H*d] (the Q input reinterpreted)
+    and SwiGLU on [B*N, 13824] (the pages give no MLP width; 13824 is read
+    for a 5120-wide SwiGLU block).  HBM-bound: GB/s against the measured copy
+    bandwidth.  Not part of the timed step."""
+    import torch
+
+    C = wl.H * wl.d
+    hid = x["q"].view(wl.B, wl.N, C)
+    g = torch.Generator(device=dev).manual_seed(11)
+    shift = (torch.randn((wl.B, C), generator=g, device=dev) * 0.5).to(torch.bfloat16)
+    scale = (torch.randn((wl.B, C), generator=g, device=dev) * 0.3).to(torch.bfloat16)
+    a_out = torch.empty_like(hid)
+    F = 13824
+    rows = wl.B * wl.N
+    gate = torch.randn((rows, F), generator=g, device=dev).to(torch.bfloat16)
+    up = torch.randn((rows, F), generator=g, device=dev).to(torch.bfloat16)
+    s_out = torch.empty_like(gate)
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record()
+        for _ in range(iters):
+            fn()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / iters
+
+    a_ms = timed(lambda: sb.adaln_modulate(hid, shift, scale, out=a_out))
+    s_ms = timed(lambda: sb.swiglu(gate, up, out=s_out))
+    a_bytes = 2.0 * rows * C * 2 + 2.0 * wl.B * C * 2
+    s_bytes = 3.0 * rows * F * 2
+    res = {}
+    for key, ms, nbytes, shape in (("adaln", a_ms, a_bytes, [wl.B, wl.N, C]), ("swiglu", s_ms, s_bytes, [rows, F])):
+        gbps = nbytes / (ms * 1e-3) / 1e9
+        res[key] = {"ms": round(ms, 4), "gbps": round(gbps, 1), "frac_of_hbm": round(gbps / peaks["hbm_gbs"], 4),
+                    "shape": shape, "bytes": nbytes}
+    del gate, up, s_out, a_out
+    return res
+
+
 def run_ours(args):
     import torch
 
@@ -370,6 +416,7 @@ def run_ours(args):
             del lw
 
     peaks = measured_peaks()
+    dit = None if args.no_dit else measure_dit_ops(sb, x, wl, dev, peaks)
     attn_tflops = flops / (att_ms * 1e-3) / 1e12
     pro_bytes = 4.0 * wl.B * wl.N * wl.H * wl.d * 2 + 2.0 * wl.B * wl.H * wl.nblk * wl.d * 4
     sel_bytes = 2.0 * wl.B * wl.H * wl.nblk * wl.d * 4 + wl.B * wl.H * wl.nblk * (K + 1) * 4
@@ -392,6 +439,8 @@ def run_ours(args):
             "gpu_launches": layer.launches_per_call * args.steps, "clocks": clk}
     if e2e is not None:
         line["e2e"] = e2e
+    if dit is not None:
+        line.update(dit)
     if sweep:
         line["sweep"] = sweep
 

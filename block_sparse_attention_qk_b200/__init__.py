@@ -2,10 +2,10 @@
 SubBlock block selection and block-sparse attention, behind a C ABI
 (include/sbattn.h) with a thin torch binding."""
 
-from .api import (AttentionLayer, SBAttnError, attention_flops, forward, keep_count, nblocks,  # noqa: F401
-                  qk_norm_rope, select_blocks, select_blocks_pooled, select_blocks_threshold,
-                  select_workspace_bytes)
+from .api import (AttentionLayer, SBAttnError, adaln_modulate, attention_flops, forward, keep_count,  # noqa: F401
+                  nblocks, qk_norm_rope, select_blocks, select_blocks_pooled, select_blocks_threshold,
+                  select_workspace_bytes, swiglu)
 
-__all__ = ["AttentionLayer", "SBAttnError", "attention_flops", "forward", "keep_count", "nblocks",
-           "qk_norm_rope", "select_blocks", "select_blocks_pooled", "select_blocks_threshold",
-           "select_workspace_bytes"]
+__all__ = ["AttentionLayer", "SBAttnError", "adaln_modulate", "attention_flops", "forward", "keep_count",
+           "nblocks", "qk_norm_rope", "select_blocks", "select_blocks_pooled", "select_blocks_threshold",
+           "select_workspace_bytes", "swiglu"]

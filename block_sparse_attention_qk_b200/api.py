@@ -170,6 +170,49 @@ def forward(q_rot, k_rot, v, kept_idx, kept_cnt, *, scale=None, out=None, status
     return out
 
 
+def adaln_modulate(x, shift, scale, *, eps=1e-6, out=None):
+    """AdaLN of x [B, N, C] bf16 with per-sample shift, scale [B, C] bf16:
+    LayerNorm (no affine) * (1 + scale) + shift; returns bf16 [B, N, C]."""
+    _act("x", x), _act("shift", shift), _act("scale", scale)
+    B, N, C = x.shape
+    if tuple(shift.shape) != (B, C) or tuple(scale.shape) != (B, C):
+        raise ValueError("shift and scale must be [B, C]")
+    out = torch.empty_like(x) if out is None else _act("out", out)
+    rc = lib().sbattn_adaln_modulate(_ptr(x), _ptr(shift), _ptr(scale), _ptr(out), B, N, C, float(eps),
+                                     _stream(x.device))
+    _check("sbattn_adaln_modulate", rc)
+    return out
+
+
+def swiglu(gate, up=None, *, out=None):
+    """silu(gate) * up.  With up=None, gate is a fused [rows, 2F] projection
+    output whose first F columns are the gate and the last F the up half.
+    Returns bf16 [rows, F]."""
+    if up is None:
+        h = _act("gate_up", gate)
+        rows, two_f = h.reshape(-1, h.shape[-1]).shape
+        if two_f % 2:
+            raise ValueError("the fused projection output needs an even last dimension")
+        F, ld = two_f // 2, two_f
+        g_ptr = h.data_ptr()
+        u_ptr = g_ptr + F * h.element_size()
+        lead = h.shape[:-1]
+        dev = h.device
+    else:
+        _act("gate", gate), _act("up", up)
+        if gate.shape != up.shape:
+            raise ValueError("gate and up must have the same shape")
+        F = gate.shape[-1]
+        rows, ld = gate.numel() // F, F
+        g_ptr, u_ptr = gate.data_ptr(), up.data_ptr()
+        lead = gate.shape[:-1]
+        dev = gate.device
+    out = torch.empty(tuple(lead) + (F,), device=dev, dtype=torch.bfloat16) if out is None else _act("out", out)
+    rc = lib().sbattn_swiglu(ctypes.c_void_p(g_ptr), ctypes.c_void_p(u_ptr), _ptr(out), rows, F, ld, _stream(dev))
+    _check("sbattn_swiglu", rc)
+    return out
+
+
 class AttentionLayer:
     """The whole hot path of one attention layer with preallocated device
     buffers: prologue (with fused block pooling) -> selection -> attention.

@@ -22,7 +22,7 @@ INCLUDE_DIR = os.path.join(ROOT, "include")
 OUT_DIR = os.path.join(HERE, "lib")
 LIB_PATH = os.path.join(OUT_DIR, "libsbattn.so")
 
-SOURCES = ["api.cu", "prologue.cu", "select.cu", "attention.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "prologue.cu", "select.cu", "attention.cu", "noalloc.cu", "dit_ops.cu"]
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH_FLAGS + [
     "-O3", "-lineinfo", "-std=c++17",

@@ -214,4 +214,29 @@ SBATTN_API int sbattn_forward(const uint16_t* q_rot, const uint16_t* k_rot, cons
   return launch_attention(a, static_cast<cudaStream_t>(stream));
 }
 
+SBATTN_API int sbattn_adaln_modulate(const uint16_t* x, const uint16_t* shift, const uint16_t* scale,
+                                     uint16_t* out, int B, int N, int C, float eps, void* stream) {
+  if (!x || !shift || !scale || !out) return SBATTN_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || C < 1 || !(isfinite(eps) && eps >= 0.f)) return SBATTN_ERR_INVALID_ARG;
+  if ((long long)B * N * C > (1ll << 40)) return SBATTN_ERR_INVALID_ARG;
+  if (C % 8 != 0 || C > kMaxAdaLNChannels) return SBATTN_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(x) || !aligned16(shift) || !aligned16(scale) || !aligned16(out)) return SBATTN_ERR_MISALIGNED;
+  DitArgs a{};
+  a.x = x; a.shift = shift; a.scale = scale; a.out = out;
+  a.B = B; a.N = N; a.C = C; a.eps = eps;
+  return launch_adaln(a, static_cast<cudaStream_t>(stream));
+}
+
+SBATTN_API int sbattn_swiglu(const uint16_t* gate, const uint16_t* up, uint16_t* out, int64_t rows, int F,
+                             int64_t ld_in, void* stream) {
+  if (!gate || !up || !out) return SBATTN_ERR_INVALID_ARG;
+  if (rows < 1 || F < 8 || F % 8 != 0 || ld_in < F || ld_in % 8 != 0) return SBATTN_ERR_INVALID_ARG;
+  if (rows > (1ll << 40) / ld_in) return SBATTN_ERR_INVALID_ARG;
+  if (!aligned16(gate) || !aligned16(up) || !aligned16(out)) return SBATTN_ERR_MISALIGNED;
+  SwigluArgs a{};
+  a.gate = gate; a.up = up; a.out = out;
+  a.rows = rows; a.ld_in = ld_in; a.F = F;
+  return launch_swiglu(a, static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

@@ -25,6 +25,26 @@ size_t prologue_table_bytes(int T, int Hh, int W, int dim_t, int dim_h, int dim_
 int launch_prologue(const PrologueArgs& a, cudaStream_t stream);
 int launch_pool(const PrologueArgs& a, cudaStream_t stream);
 
+struct DitArgs {  // AdaLN modulation
+  const uint16_t* x;      // [B, N, C]
+  const uint16_t* shift;  // [B, C]
+  const uint16_t* scale;  // [B, C]
+  uint16_t* out;          // [B, N, C]
+  int B, N, C;
+  float eps;
+};
+constexpr int kMaxAdaLNChannels = 6144;
+int launch_adaln(const DitArgs& a, cudaStream_t stream);
+
+struct SwigluArgs {
+  const uint16_t* gate;  // row r at gate + r * ld_in
+  const uint16_t* up;
+  uint16_t* out;         // [rows, F]
+  long rows, ld_in;
+  int F;
+};
+int launch_swiglu(const SwigluArgs& a, cudaStream_t stream);
+
 struct SelectArgs {
   const float* q_bar;  // [B, H, nblk, d]
   const float* k_bar;

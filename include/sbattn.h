@@ -212,6 +212,40 @@ SBATTN_API int sbattn_forward(const uint16_t* q_rot, const uint16_t* k_rot, cons
                               uint16_t* out, int B, int N, int H, int d,
                               float softmax_scale, int32_t* status, void* stream);
 
+/* ---- 4. fused DiT-block elementwise steps around attention -------------
+ * [p3] "先把近两倍的免费收益拿走": the lossless gain also comes from fused
+ * AdaLN and SwiGLU kernels (fewer intermediate tensors, memory passes and
+ * launches).  The page names the operations only; these are the standard
+ * DiT definitions.
+ *
+ * AdaLN: for every token row x (C channels) of sample b,
+ *     y = (x - mean(x)) / sqrt(var(x) + eps) * (1 + scale_b) + shift_b
+ * with the biased (1/C) variance and no learned LayerNorm affine; shift and
+ * scale are the per-sample conditioning vectors.  One pass: fp32 statistics
+ * and arithmetic, output rounded to bf16 (nearest even).
+ *
+ *   x            [B, N, C] bf16 input
+ *   shift, scale [B, C] bf16 conditioning vectors
+ *   out          [B, N, C] bf16 output; may alias x (in place)
+ *   C            a multiple of 8, at most 6144 (a row is held in registers)
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (C), MISALIGNED, CUDA.
+ */
+SBATTN_API int sbattn_adaln_modulate(const uint16_t* x, const uint16_t* shift, const uint16_t* scale,
+                                     uint16_t* out, int B, int N, int C, float eps, void* stream);
+
+/* SwiGLU: out[r, f] = silu(gate[r, f]) * up[r, f], silu(a) = a / (1 + e^-a),
+ * fp32 arithmetic, output rounded to bf16 (nearest even).
+ *
+ *   gate, up     bf16 rows of F elements, row r at gate + r * ld_in (the two
+ *                halves of a fused [rows, 2F] projection output have
+ *                ld_in = 2F and up = gate + F; separate tensors ld_in = F)
+ *   out          [rows, F] bf16, contiguous; must not overlap gate / up
+ *   F, ld_in     multiples of 8, ld_in >= F
+ * Errors: INVALID_ARG, MISALIGNED, CUDA.
+ */
+SBATTN_API int sbattn_swiglu(const uint16_t* gate, const uint16_t* up, uint16_t* out,
+                             int64_t rows, int F, int64_t ld_in, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

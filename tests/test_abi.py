@@ -163,6 +163,37 @@ def test_forward_validation(L):
     assert _forward(L, B=1 << 20, N=1 << 20, H=1 << 10) == SHAPE  # item count overflows int32
 
 
+def _adaln(L, x=A, shift=A + 0x1000, scale=A + 0x2000, out=A + 0x100000, B=2, N=300, C=5120, eps=1e-6):
+    return L.sbattn_adaln_modulate(x, shift, scale, out, B, N, C, eps, None)
+
+
+def test_adaln_validation(L):
+    assert _adaln(L, x=None) == INVALID
+    assert _adaln(L, shift=None) == INVALID
+    assert _adaln(L, N=0) == INVALID
+    assert _adaln(L, eps=float("nan")) == INVALID
+    assert _adaln(L, eps=-1.0) == INVALID
+    assert _adaln(L, C=5124) == SHAPE          # not a multiple of 8
+    assert _adaln(L, C=8192) == SHAPE          # more channels than a warp holds
+    assert _adaln(L, scale=A + 0x2008) == MISALIGNED
+    assert _adaln(L, out=A + 4) == MISALIGNED
+
+
+def _swiglu(L, gate=A, up=A + 0x10000, out=A + 0x100000, rows=100, F=13824, ld=13824):
+    return L.sbattn_swiglu(gate, up, out, rows, F, ld, None)
+
+
+def test_swiglu_validation(L):
+    assert _swiglu(L, up=None) == INVALID
+    assert _swiglu(L, rows=0) == INVALID
+    assert _swiglu(L, F=12) == INVALID          # not a multiple of 8
+    assert _swiglu(L, ld=13816) == INVALID      # row stride shorter than a row
+    assert _swiglu(L, ld=13828) == INVALID      # row stride not a multiple of 8
+    assert _swiglu(L, rows=1 << 40) == INVALID  # size overflow
+    assert _swiglu(L, gate=A + 8) == MISALIGNED
+    assert _swiglu(L, out=A + 0x100002) == MISALIGNED
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU failure path")
 def test_valid_call_without_gpu_fails_cleanly(L):
     # every argument is valid, so the call reaches the CUDA runtime, which
