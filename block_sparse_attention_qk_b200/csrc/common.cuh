@@ -58,19 +58,6 @@ SB_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
-// Non-blocking test of the phase with the given parity.
-SB_DEV bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-
 // try_wait with a suspend-time hint: the waiting thread sleeps in hardware
 // until the phase completes or about `hint_ns` pass, instead of spinning on
 // issue slots that the other warps of its SM sub-partition need.
@@ -239,29 +226,6 @@ SB_DEV uint64_t f2_mul(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
-// 2^x for two lanes on the FMA pipe instead of the MUFU unit, for finite
-// x <= 126 (x below -125 is not supported): x = j + f with j = rint(x) and
-// |f| <= 1/2, 2^f by its Taylor series to degree 4 (coefficients ln2^k / k!;
-// relative error below 6e-5, far under bf16 rounding), and j added to the
-// exponent field.  Adding 1.5 * 2^23 rounds x to an integer held in the low
-// mantissa bits of y, so (bits(y) << 23) is j in the exponent position.
-SB_DEV void exp2_poly_x2(float x0, float x1, float& r0, float& r1) {
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  const uint64_t xx = f2_pack(x0, x1);
-  const uint64_t y = f2_add(xx, f2_pack(kMagic, kMagic));
-  const uint64_t jf = f2_add(y, f2_pack(-kMagic, -kMagic));
-  const uint64_t f = f2_fma(jf, f2_pack(-1.0f, -1.0f), xx);
-  uint64_t p = f2_fma(f2_pack(0.0096181291f, 0.0096181291f), f, f2_pack(0.0555041087f, 0.0555041087f));
-  p = f2_fma(p, f, f2_pack(0.2402265070f, 0.2402265070f));
-  p = f2_fma(p, f, f2_pack(0.6931471806f, 0.6931471806f));
-  p = f2_fma(p, f, f2_pack(1.0f, 1.0f));
-  float p0, p1, y0, y1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(y, y0, y1);
-  r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(y0) << 23));
-  r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(y1) << 23));
-}
-
 // max of three fp32 values in one instruction (sm_100)
 SB_DEV float fmax3(float a, float b, float c) {
   float r;
@@ -269,8 +233,5 @@ SB_DEV float fmax3(float a, float b, float c) {
   return r;
 }
 
-SB_DEV void named_barrier_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 }  // namespace sbattn
