@@ -26,11 +26,12 @@
 // streams interleave in the tensor pipe.  TMA streaming and MMAs on the same
 // SM do not slow each other down.
 //
-// Shared memory: Q (one stage), K and V (three stages each, so that a copy
-// has time to land while two tiles are in compute) and one P^T buffer
-// released in two key halves: the softmax threads of key rows 0-63 may write
-// the next P^T as soon as the first four PV K-steps are done, and the PV
-// issuer waits for the second half only before the last four.
+// Shared memory (208 KB): Q (one stage), K (three stages), V (two) and two
+// P^T buffers, each released in two key halves: the softmax threads of key
+// rows 0-63 may refill a buffer as soon as the first four PV K-steps that
+// read it are done, and the PV issuer waits for the second half only before
+// the last four.  The softmax threads make their P^T stores visible to the
+// tensor core with one async-proxy fence per step.
 //
 // Two softmax work-groups of 128 threads split the 64 query columns of every
 // tile (32 each); a thread owns one TMEM lane, i.e. one KEY row across its 32
