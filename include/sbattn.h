@@ -202,8 +202,11 @@ SBATTN_API int sbattn_select_blocks_noalloc(const uint16_t* q_rot, const uint16_
  *   status          optional device int32 (may be NULL).  If given, the
  *                   kernel stores a nonzero SBATTN_ERR_* code there when a
  *                   kept index or count is out of range (that block/row is
- *                   skipped) or a bounded internal wait runs out; it never
- *                   clears it.  Zero it before the call and read it after the
+ *                   skipped; DEVICE), when a logit exceeds the row's running
+ *                   maximum by more than 100 in log2 units before the
+ *                   maximum is raised (its weight 2^x could overflow the
+ *                   sums; DEVICE), or when a bounded internal wait runs out
+ *                   (TIMEOUT); it never clears it.  Zero it before the call and read it after the
  *                   stream has reached the call.
  * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (d != 128), MISALIGNED, CUDA.
  */
