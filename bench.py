@@ -269,7 +269,9 @@ def config_of(wl, K, n_gpus):
             "B": wl.B, "H": wl.H, "head_dim": wl.d, "grid": [wl.T, wl.Hh, wl.W], "N": wl.N, "nblk": wl.nblk,
             "sparsity": wl.sparsity, "kept_blocks": K, "kept_fraction": K / wl.nblk,
             "parallelism": f"{n_gpus} independent replicas" if n_gpus > 1 else "single GPU",
-            "l2_policy": "inputs (3 x B*N*H*d bf16) larger than the 126 MB L2; no flush"}
+            "l2_policy": ("inputs (3 x B*N*H*d bf16) larger than the 126 MB L2; no flush"
+                          if 3 * wl.B * wl.N * wl.H * wl.d * 2 > 126e6 else
+                          "inputs smaller than the 126 MB L2: timed cache-warm (a test size, not a bench line)")}
 
 
 def measure_dit_ops(sb, x, wl, dev, peaks, iters=5):
