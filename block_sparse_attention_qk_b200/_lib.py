@@ -14,6 +14,7 @@ _c_int, _c_double, _c_float, _c_size, _c_void = ctypes.c_int, ctypes.c_double, c
 SIGNATURES = {
     "sbattn_strerror": (ctypes.c_char_p, [_c_int]),
     "sbattn_version": (_c_int, []),
+    "sbattn_check_status": (_c_int, [_c_void, _c_void]),
     "sbattn_keep_count": (_c_int, [_c_int, _c_double, ctypes.POINTER(_c_int)]),
     "sbattn_select_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
     "sbattn_qk_norm_rope": (_c_int, [_c_void] * 8 + [_c_int] * 9 + [_c_float, _c_float, _c_void]),

@@ -47,6 +47,17 @@ def _act(name, t, dtype=torch.bfloat16):
     return t
 
 
+def check_status(status=None, device=None) -> None:
+    """Synchronise the current stream and raise SBAttnError if a CUDA error
+    surfaced or a kernel stored an error code in `status` (an int32 CUDA
+    tensor of one element, as passed to `forward`)."""
+    if status is not None:
+        _act("status", status, torch.int32)
+        device = status.device
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    _check("sbattn_check_status", lib().sbattn_check_status(_ptr(status), _stream(dev)))
+
+
 def nblocks(N: int) -> int:
     return -(-N // BLOCK)
 
@@ -309,9 +320,7 @@ class AttentionLayer:
 
     def check_status(self):
         """Synchronise and raise if a kernel recorded a device-side error."""
-        code = int(self.status.item())
-        if code != 0:
-            raise SBAttnError("device status", code)
+        check_status(self.status)
 
 
 def attention_flops(B, N, H, K, d=HEAD_DIM) -> float:

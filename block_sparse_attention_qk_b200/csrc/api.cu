@@ -7,8 +7,6 @@
 
 namespace sbattn {
 
-namespace {
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int nblk_of(long long N) { return (int)((N + kBlock - 1) / kBlock); }
@@ -22,6 +20,15 @@ int check_dims(long long B, long long N, long long H, long long d) {
   if (N > 0x7FFFFFFFLL - kBlock) return SBATTN_ERR_UNSUPPORTED_SHAPE;
   return SBATTN_OK;
 }
+
+// Output checks shared by every selection entry point.
+int check_select_outputs(const int32_t* kept_idx, const int32_t* kept_cnt, const float* scores) {
+  if (!kept_idx || !kept_cnt) return SBATTN_ERR_INVALID_ARG;
+  if (!aligned16(kept_idx) || !aligned16(kept_cnt) || (scores && !aligned16(scores))) return SBATTN_ERR_MISALIGNED;
+  return SBATTN_OK;
+}
+
+namespace {
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -80,6 +87,24 @@ SBATTN_API const char* sbattn_strerror(int status) {
   }
 }
 
+SBATTN_API int sbattn_check_status(const int32_t* status, void* stream) {
+  if (status != nullptr && (reinterpret_cast<uintptr_t>(status) & 3u)) return SBATTN_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();  // clear a non-sticky error so that later calls start clean
+    return SBATTN_ERR_CUDA;
+  }
+  if (status == nullptr) return SBATTN_OK;
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, status, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return SBATTN_ERR_CUDA;
+  }
+  if (v == SBATTN_OK) return SBATTN_OK;
+  return (v >= SBATTN_ERR_INVALID_ARG && v <= SBATTN_ERR_CAPACITY) ? v : SBATTN_ERR_DEVICE;
+}
+
 SBATTN_API int sbattn_version(void) { return 1 * 10000 + 0 * 100 + 0; }
 
 SBATTN_API int sbattn_keep_count(int nblk, double sparsity, int* K_out) {
@@ -122,12 +147,6 @@ SBATTN_API int sbattn_qk_norm_rope(const uint16_t* q, const uint16_t* k, const u
   a.B = B; a.N = (int)N; a.H = H; a.T = T; a.Hh = Hh; a.W = W; a.nblk = nblk_of(N);
   a.dim_t = dim_t; a.dim_h = dim_h; a.dim_w = dim_w; a.theta = theta; a.eps = eps;
   return launch_prologue(a, static_cast<cudaStream_t>(stream));
-}
-
-static int check_select_outputs(int32_t* kept_idx, int32_t* kept_cnt, float* scores) {
-  if (!kept_idx || !kept_cnt) return SBATTN_ERR_INVALID_ARG;
-  if (!aligned16(kept_idx) || !aligned16(kept_cnt) || (scores && !aligned16(scores))) return SBATTN_ERR_MISALIGNED;
-  return SBATTN_OK;
 }
 
 SBATTN_API int sbattn_select_blocks_pooled(const float* q_bar, const float* k_bar, int B, int nblk, int H, int d,

@@ -30,8 +30,10 @@
 // P^T buffers, each released in two key halves: the softmax threads of key
 // rows 0-63 may refill a buffer as soon as the first four PV K-steps that
 // read it are done, and the PV issuer waits for the second half only before
-// the last four.  The softmax threads make their P^T stores visible to the
-// tensor core with one async-proxy fence per step.
+// the last four.  The PV issuer, after acquiring a half through its
+// mbarrier, executes the async-proxy fence that makes the softmax threads'
+// generic stores visible to the tensor core (the fence may sit anywhere on
+// the release/acquire path from the stores to the MMA that reads them).
 //
 // Two softmax work-groups of 128 threads split the 64 query columns of every
 // tile (32 each); a thread owns one TMEM lane, i.e. one KEY row across its 32
@@ -436,6 +438,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                (!first || mbar_wait(&ms->o_empty, (ts.n & 1) ^ 1, abort_flag));
           if (!ok) break;
           tc_fence_after();
+          // the softmax threads' P^T stores (generic proxy), acquired through
+          // p_full, become visible to the tensor core (async proxy)
+          fence_proxy_async_smem();
           const uint64_t vd = smem_desc(sbase + kOffV + vs * kKVBytes, 16384, 1024, kSwizzle128B);
           const uint64_t pd = smem_desc(sbase + kOffP + pb * kPBytes, 8192, 1024, kSwizzle128B);
           // K-step kk accumulates into partial kk mod 4; the first tile of an
@@ -446,6 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(&ms->p_empty[pb][0]);  // key rows 0-63 of this P^T buffer are free again
           if (!(ok = mbar_wait(&ms->p_full[pb][1], pph, abort_flag))) break;
           tc_fence_after();
+          fence_proxy_async_smem();
 #pragma unroll
           for (int kk = 4; kk < 8; ++kk)
             umma_bf16(tmem + kColO + (kk & 3) * 64, vd + (uint64_t)(kk * 128), pd + (uint64_t)(kk * 128), kIdescPV, 1u);
@@ -668,9 +674,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 make_uint4(pk[tile][4 * c4], pk[tile][4 * c4 + 1], pk[tile][4 * c4 + 2], pk[tile][4 * c4 + 3]);
         }
         if (!ok) break;
-        // one proxy fence per step: it is cheap alone, but costly while the
-        // SM's async proxy is busy with copies and MMAs
-        fence_proxy_async_smem();
+        // the PV issuer makes these stores visible to the tensor core after
+        // acquiring them through p_full (one proxy fence per half tile there
+        // instead of one per softmax thread and step here)
         mbar_arrive(&ms->p_full[gA % 2][half]);
         if (hasB) mbar_arrive(&ms->p_full[gB % 2][half]);
       }

@@ -58,6 +58,19 @@ SB_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
+// Non-blocking test of the phase with the given parity (never suspends).
+SB_DEV bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
 // try_wait with a suspend-time hint: the waiting thread sleeps in hardware
 // until the phase completes or about `hint_ns` pass, instead of spinning on
 // issue slots that the other warps of its SM sub-partition need.
@@ -195,6 +208,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
          | ((uint32_t)(N >> 3) << 17)   // N / 8
          | ((uint32_t)(M >> 4) << 24);  // M / 16
 }
+
+// Register reallocation between warpgroups (all four warps of a warpgroup
+// execute the same instruction): give registers back / take them from the
+// pool the CTA was launched with.
+template <uint32_t kRegs>
+SB_DEV void warpgroup_regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegs) : "memory"); }
+template <uint32_t kRegs>
+SB_DEV void warpgroup_regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegs) : "memory"); }
 
 // ------------------------------------------------------------- misc math --
 

@@ -5,6 +5,12 @@
 
 namespace sbattn {
 
+// Host-side argument checks shared by the entry points (api.cu).
+bool aligned16(const void* p);
+int nblk_of(long long N);
+int check_dims(long long B, long long N, long long H, long long d);
+int check_select_outputs(const int32_t* kept_idx, const int32_t* kept_cnt, const float* scores);
+
 struct PrologueArgs {
   const uint16_t* q;   // input rows (prologue: raw Q; pooling: rotated Q)
   const uint16_t* k;

@@ -69,6 +69,21 @@ extern "C" {
 /* Human-readable name of a status code (static string, never NULL). */
 SBATTN_API const char* sbattn_strerror(int status);
 
+/* Waits until `stream` has finished all work queued on it so far, then
+ * reports the first error found (this call synchronises; use it in tests,
+ * debug paths or at the end of a step, not inside a timed loop):
+ *   SBATTN_ERR_CUDA  an asynchronous CUDA error surfaced (a failed kernel);
+ *   the nonzero code a kernel stored in the device status word `status`
+ *                    (SBATTN_ERR_DEVICE or SBATTN_ERR_TIMEOUT, see
+ *                    sbattn_forward), read back with one 4-byte copy on
+ *                    `stream`;
+ *   SBATTN_OK        otherwise.
+ *   status   optional device int32 (NULL: only the stream is checked); it is
+ *            read, not cleared.  4-byte aligned, else MISALIGNED.
+ * The library keeps no global error state: the status word is the caller's.
+ */
+SBATTN_API int sbattn_check_status(const int32_t* status, void* stream);
+
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 SBATTN_API int sbattn_version(void);
 
@@ -164,18 +179,26 @@ SBATTN_API int sbattn_select_blocks_threshold(const float* q_bar, const float* k
  * for such callers.
  *
  * The pooled block means live in a fixed scratch array compiled into the
- * library (4 MiB of device memory, held on every GPU that loads the library
- * until the process exits), so the call allocates nothing and takes no
- * workspace.  Limit: B * H * ceil(N/64) <= SBATTN_NOALLOC_MAX_POOLED_ROWS;
- * larger problems are rejected with SBATTN_ERR_WORKSPACE before anything is
- * launched (use sbattn_select_blocks with a workspace for them).
+ * library (4 MiB of device memory, held until the process exits), so the
+ * call allocates nothing and takes no workspace.  Limit: B * H * ceil(N/64)
+ * <= SBATTN_NOALLOC_MAX_POOLED_ROWS; larger problems are rejected with
+ * SBATTN_ERR_WORKSPACE before anything is launched (use sbattn_select_blocks
+ * with a workspace for them).
  *
- * The first call on each device looks up that device's address of the
- * scratch array (with that device current); make that first call before any
- * stream capture.  All calls on a device share the one array and each call
- * overwrites every value it reads, so nothing needs clearing between calls;
- * but calls whose work overlaps on the GPU (different streams, or different
- * host threads, without ordering between them) race on it.
+ * Warm-up: the first call in each context looks up that device's address of
+ * the array (with the device current).  Under CUDA's lazy module loading
+ * (the default) that lookup is also what loads the library module holding
+ * the array, so the first call on a device is the one that creates its
+ * 4 MiB; until then the array does not exist on that device.  Make one call
+ * on every device before the point where allocation becomes forbidden, and
+ * before any stream capture.  The address is cached per device and looked up
+ * again when the device's current context changes (after cudaDeviceReset or
+ * when another context is made current).
+ *
+ * All calls on a device share the one array and each call overwrites every
+ * value it reads, so nothing needs clearing between calls; but calls whose
+ * work overlaps on the GPU (different streams, or different host threads,
+ * without ordering between them) race on it.
  * Other arguments, outputs and errors as for sbattn_select_blocks.
  */
 #define SBATTN_NOALLOC_MAX_POOLED_ROWS 4096

@@ -30,6 +30,12 @@ int main(void) {
   if (sbattn_adaln_modulate(NULL, NULL, NULL, NULL, 1, 1, 8, 1e-6f, NULL) != SBATTN_ERR_INVALID_ARG) return 6;
   if (sbattn_swiglu(NULL, NULL, NULL, 1, 8, 8, NULL) != SBATTN_ERR_INVALID_ARG) return 7;
   if (sbattn_select_workspace_bytes(1, 124992, 40, 128) != (size_t)2 * 40 * 1953 * 128 * 4) return 8;
+  /* the status path: a misaligned status word is rejected before any CUDA
+     call; with no status word the call only checks the stream, which on a
+     machine without a GPU reports a CUDA error instead of crashing */
+  if (sbattn_check_status((const int32_t*)(uintptr_t)0x1002, NULL) != SBATTN_ERR_MISALIGNED) return 9;
+  rc = sbattn_check_status(NULL, NULL);
+  if (rc != SBATTN_OK && rc != SBATTN_ERR_CUDA) { printf("check_status rc=%d\n", rc); return 10; }
   printf("c abi ok\n");
   return 0;
 }

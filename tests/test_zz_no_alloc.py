@@ -80,6 +80,48 @@ def test_no_alloc_selection_matches_workspace_entry_point_twice_in_a_row():
         assert torch.all(got[1] == K)
 
 
+def test_no_alloc_selection_at_exactly_the_scratch_limit():
+    """B * H * nblk == 4096: the pooled key means end at the last byte of the
+    built-in array, so an off-by-one in the limit or the offsets would show."""
+    sb_build.build()
+    L = lib()
+    wl = custom_workload("edge", B=1, H=64, T=1, Hh=64, W=64, sparsity=0.75, seed=33)  # N = 4096, nblk = 64
+    assert wl.B * wl.H * wl.nblk == MAX_ROWS
+    q, k = _rotated(wl)
+    ref, got = _run_both(L, q, k, wl.sparsity)
+    assert torch.equal(got[2], ref[2])
+    assert torch.equal(got[0], ref[0])
+    assert torch.equal(got[1], ref[1])
+
+
+def test_no_alloc_calls_allocate_no_device_memory_after_the_first():
+    """After one warm-up call on the device (which, under CUDA's lazy module
+    loading, is when the library's built-in array comes into existence),
+    further calls leave the device's free memory unchanged."""
+    sb_build.build()
+    L = lib()
+    wl = custom_workload("mem", B=1, H=4, T=2, Hh=16, W=32, sparsity=0.5, seed=34)
+    q, k = _rotated(wl)
+    B, N, H, d = q.shape
+    nblk = -(-N // 64)
+    K = orc.keep_count(nblk, wl.sparsity)
+    out = _outputs(B, H, nblk, K)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+    def call():
+        rc = L.sbattn_select_blocks_noalloc(_p(q), _p(k), B, N, H, d, wl.sparsity, _p(out[0]), _p(out[1]), K,
+                                            _p(out[2]), stream)
+        assert rc == 0
+
+    call()  # warm-up
+    torch.cuda.synchronize()
+    free_before = torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free_before
+
+
 def test_no_alloc_rejects_problems_beyond_the_scratch():
     sb_build.build()
     L = lib()
