@@ -28,6 +28,9 @@ SIGNATURES = {
                                               _c_void, _c_void, _c_int, _c_void, _c_void]),
     "sbattn_forward": (_c_int, [_c_void, _c_void, _c_void, _c_void, _c_void, _c_int, _c_void,
                                 _c_int, _c_int, _c_int, _c_int, _c_float, _c_void, _c_void]),
+    "sbattn_forward_diag": (_c_int, [_c_void, _c_void, _c_void, _c_void, _c_void, _c_int, _c_void,
+                                     _c_int, _c_int, _c_int, _c_int, _c_float, _c_void, ctypes.c_ulonglong, _c_int,
+                                     _c_void]),
     "sbattn_adaln_modulate": (_c_int, [_c_void, _c_void, _c_void, _c_void, _c_int, _c_int, _c_int, _c_float,
                                        _c_void]),
     "sbattn_swiglu": (_c_int, [_c_void, _c_void, _c_void, ctypes.c_int64, _c_int, ctypes.c_int64, _c_void]),

@@ -228,9 +228,13 @@ class AttentionLayer:
     """The whole hot path of one attention layer with preallocated device
     buffers: prologue (with fused block pooling) -> selection -> attention.
 
-    `__call__` takes device or host tensors; host tensors are copied in (and
-    the output copied back) on the current stream, which is what an
-    end-to-end caller with host buffers pays.
+    `run_device` takes tensors already on the GPU.  `__call__` also takes
+    host tensors (pinned, for asynchronous copies): then each call copies its
+    inputs in and its output back, pipelined over two input/output slots so
+    that the host-to-device copy of call i + 1 and the device-to-host copy of
+    call i - 1 run on their own streams while call i computes.  The output
+    host tensor of a call is complete once `drain()` (or a device
+    synchronisation) follows it.
     """
 
     def __init__(self, B, T, Hh, W, H, sparsity, *, device="cuda", dims=(32, 48, 48), theta=10000.0,
@@ -242,16 +246,11 @@ class AttentionLayer:
         self.fused_pool = fused_pool
         self.K = keep_count(self.nblk, sparsity)
         dev = torch.device(device)
-        shp = (B, self.N, H, HEAD_DIM)
         self.dev = dev
-        self.q_in = torch.empty(shp, device=dev, dtype=torch.bfloat16)
-        self.k_in = torch.empty_like(self.q_in)
-        self.v_in = torch.empty_like(self.q_in)
-        self.wq_in = torch.empty((HEAD_DIM,), device=dev, dtype=torch.bfloat16)
-        self.wk_in = torch.empty_like(self.wq_in)
-        self.q_rot = torch.empty_like(self.q_in)
-        self.k_rot = torch.empty_like(self.q_in)
-        self.out = torch.empty_like(self.q_in)
+        self.shape = (B, self.N, H, HEAD_DIM)
+        self.q_rot = torch.empty(self.shape, device=dev, dtype=torch.bfloat16)
+        self.k_rot = torch.empty_like(self.q_rot)
+        self.out = torch.empty_like(self.q_rot)
         self.q_bar = torch.empty((B, H, self.nblk, HEAD_DIM), device=dev, dtype=torch.float32)
         self.k_bar = torch.empty_like(self.q_bar)
         self.kept_idx = torch.empty((B, H, self.nblk, self.K), device=dev, dtype=torch.int32)
@@ -259,15 +258,19 @@ class AttentionLayer:
         self.status = torch.zeros((1,), device=dev, dtype=torch.int32)
         self.workspace = None if fused_pool else torch.empty(
             select_workspace_bytes(B, self.N, H), device=dev, dtype=torch.uint8)
+        self._slots = None  # device input/output slots of the host-buffer path (allocated on first use)
+        self._calls = 0
 
-    def run_device(self, q, k, v, w_q, w_k, events=None):
-        """Run the path on device tensors already resident in HBM.
+    def run_device(self, q, k, v, w_q, w_k, events=None, out=None):
+        """Run the path on device tensors already resident in HBM; returns the
+        output (`out` if given, else the layer's own output buffer).
 
         events: optional 4 CUDA events, recorded on the launching stream
         before the prologue, before the selection, before the attention and
         after it (per-kernel device timing)."""
         L, s = lib(), _stream(self.dev)
         B, N, H, d = self.B, self.N, self.H, HEAD_DIM
+        out = self.out if out is None else out
         if events is not None:
             events[0].record()
         if self.fused_pool:
@@ -295,28 +298,64 @@ class AttentionLayer:
         if events is not None:
             events[2].record()
         rc = L.sbattn_forward(_ptr(self.q_rot), _ptr(self.k_rot), _ptr(v), _ptr(self.kept_idx),
-                              _ptr(self.kept_cnt), self.K, _ptr(self.out), B, N, H, d, 0.0,
+                              _ptr(self.kept_cnt), self.K, _ptr(out), B, N, H, d, 0.0,
                               _ptr(self.status), s)
         _check("sbattn_forward", rc)
         if events is not None:
             events[3].record()
-        return self.out
+        return out
 
     # kernels launched per run_device call (prologue, selection [+ pooling], attention)
     @property
     def launches_per_call(self) -> int:
         return 3 if self.fused_pool else 4
 
+    def _host_slots(self):
+        if self._slots is None:
+            mk = lambda shape: torch.empty(shape, device=self.dev, dtype=torch.bfloat16)
+            self._slots = [dict(q=mk(self.shape), k=mk(self.shape), v=mk(self.shape), w_q=mk((HEAD_DIM,)),
+                                w_k=mk((HEAD_DIM,)), out=mk(self.shape),
+                                ev_in=torch.cuda.Event(), ev_done=torch.cuda.Event(), ev_out=torch.cuda.Event(),
+                                used=False)
+                           for _ in range(2)]
+            self._h2d = torch.cuda.Stream(self.dev)
+            self._d2h = torch.cuda.Stream(self.dev)
+        return self._slots
+
     def __call__(self, q, k, v, w_q, w_k, out_host=None):
         if q.is_cuda:
             return self.run_device(q, k, v, w_q, w_k)
-        for dst, src in ((self.q_in, q), (self.k_in, k), (self.v_in, v), (self.wq_in, w_q), (self.wk_in, w_k)):
-            dst.copy_(src, non_blocking=True)
-        o = self.run_device(self.q_in, self.k_in, self.v_in, self.wq_in, self.wk_in)
+        slots = self._host_slots()
+        sl = slots[self._calls % 2]
+        comp = torch.cuda.current_stream(self.dev)
+        with torch.cuda.stream(self._h2d):
+            if sl["used"]:
+                self._h2d.wait_event(sl["ev_done"])  # the slot's previous inputs have been consumed
+            for name, src in (("q", q), ("k", k), ("v", v), ("w_q", w_q), ("w_k", w_k)):
+                sl[name].copy_(src, non_blocking=True)
+            sl["ev_in"].record(self._h2d)
+        comp.wait_event(sl["ev_in"])
+        if sl["used"]:
+            comp.wait_event(sl["ev_out"])  # the slot's previous output has been read back
+        o = self.run_device(sl["q"], sl["k"], sl["v"], sl["w_q"], sl["w_k"], out=sl["out"])
+        sl["ev_done"].record(comp)
         if out_host is None:
             out_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-        out_host.copy_(o, non_blocking=True)
+        with torch.cuda.stream(self._d2h):
+            self._d2h.wait_event(sl["ev_done"])
+            out_host.copy_(o, non_blocking=True)
+            sl["ev_out"].record(self._d2h)
+        sl["used"] = True
+        self._calls += 1
         return out_host
+
+    def drain(self):
+        """Make the current stream wait for every copy issued by host-buffer
+        calls (events recorded on it afterwards include them)."""
+        if self._slots is not None:
+            comp = torch.cuda.current_stream(self.dev)
+            comp.wait_stream(self._h2d)
+            comp.wait_stream(self._d2h)
 
     def check_status(self):
         """Synchronise and raise if a kernel recorded a device-side error."""

@@ -215,9 +215,10 @@ SBATTN_API int sbattn_select_blocks(const uint16_t* q_rot, const uint16_t* k_rot
   return launch_select(a, s);
 }
 
-SBATTN_API int sbattn_forward(const uint16_t* q_rot, const uint16_t* k_rot, const uint16_t* v,
-                              const int32_t* kept_idx, const int32_t* kept_cnt, int K_capacity, uint16_t* out,
-                              int B, int N, int H, int d, float softmax_scale, int32_t* status, void* stream) {
+static int forward_impl(const uint16_t* q_rot, const uint16_t* k_rot, const uint16_t* v, const int32_t* kept_idx,
+                        const int32_t* kept_cnt, int K_capacity, uint16_t* out, int B, int N, int H, int d,
+                        float softmax_scale, int32_t* status, unsigned long long wait_limit_ns, int withhold_v_tile,
+                        void* stream) {
   if (!q_rot || !k_rot || !v || !kept_idx || !kept_cnt || !out) return SBATTN_ERR_INVALID_ARG;
   if (out == q_rot || out == k_rot || out == v) return SBATTN_ERR_INVALID_ARG;
   if (K_capacity < 1 || isnan(softmax_scale) || isinf(softmax_scale)) return SBATTN_ERR_INVALID_ARG;
@@ -230,7 +231,26 @@ SBATTN_API int sbattn_forward(const uint16_t* q_rot, const uint16_t* k_rot, cons
   a.q = q_rot; a.k = k_rot; a.v = v; a.kept_idx = kept_idx; a.kept_cnt = kept_cnt; a.out = out; a.status = status;
   a.B = B; a.N = N; a.H = H; a.nblk = nblk_of(N); a.K_capacity = K_capacity;
   a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)d);
+  a.wait_limit_ns = wait_limit_ns;
+  a.withhold_v_tile = withhold_v_tile;
   return launch_attention(a, static_cast<cudaStream_t>(stream));
+}
+
+SBATTN_API int sbattn_forward(const uint16_t* q_rot, const uint16_t* k_rot, const uint16_t* v,
+                              const int32_t* kept_idx, const int32_t* kept_cnt, int K_capacity, uint16_t* out,
+                              int B, int N, int H, int d, float softmax_scale, int32_t* status, void* stream) {
+  return forward_impl(q_rot, k_rot, v, kept_idx, kept_cnt, K_capacity, out, B, N, H, d, softmax_scale, status,
+                      kWaitLimitNs, -1, stream);
+}
+
+SBATTN_API int sbattn_forward_diag(const uint16_t* q_rot, const uint16_t* k_rot, const uint16_t* v,
+                                   const int32_t* kept_idx, const int32_t* kept_cnt, int K_capacity, uint16_t* out,
+                                   int B, int N, int H, int d, float softmax_scale, int32_t* status,
+                                   unsigned long long wait_limit_ns, int withhold_v_tile, void* stream) {
+  if (wait_limit_ns < 1000000ull || wait_limit_ns > 10ull * kWaitLimitNs) return SBATTN_ERR_INVALID_ARG;
+  if (withhold_v_tile < -1) return SBATTN_ERR_INVALID_ARG;
+  return forward_impl(q_rot, k_rot, v, kept_idx, kept_cnt, K_capacity, out, B, N, H, d, softmax_scale, status,
+                      wait_limit_ns, withhold_v_tile, stream);
 }
 
 SBATTN_API int sbattn_adaln_modulate(const uint16_t* x, const uint16_t* shift, const uint16_t* scale,

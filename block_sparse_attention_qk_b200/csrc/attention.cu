@@ -39,18 +39,17 @@
 // tile (32 each); a thread owns one TMEM lane, i.e. one KEY row across its 32
 // queries, and takes two tiles per step.  The per-query running maximum m is
 // seeded from the first step of the item (one cross-lane reduction per item).
-// Later steps need no barrier: a thread that meets a logit more than 2^8 above
-// m raises a flag and records the excess per query (atomicMax); the
-// work-group reads the flag three steps later, when the P^T ring guarantees
-// that every softmax thread has finished the flagged step, and only then --
-// rarely -- raises m (by the largest excess recorded so far) and rescales O
-// and the partial row sums.  The p values of the steps in between stay exact:
-// p up to 2^100 is fine in fp32 and bf16; a logit beyond that is reported as
-// a device error.  Each thread keeps 32 partial row sums (packed in pairs),
-// reduced once per item.  S^T of the next step is loaded from TMEM while the
-// current P^T is stored.
+// Each later step's S^T is loaded, scaled (s * scale * log2 e - m) and checked
+// one step ahead, while the previous step's P^T is stored: a thread publishes
+// per query the largest excess of its logits over m, and a work-group barrier
+// (bounded like every wait) orders all publications before the step starts.
+// When some excess passes 2^8, the group raises m by exactly that excess and
+// rescales O and the row sums before any p of the step is formed, so no p
+// exceeds 2^8 whatever the logit range.  The raise is rare in practice.  Each
+// thread keeps 32 partial row sums (packed in pairs), reduced once per item.
 //
-// Roles (384 threads, one CTA per SM, persistent over items):
+// Roles (384 threads, one CTA per SM, persistent over items; warps 0-3 run
+// with 56 registers and the softmax warps with 224 after setmaxnreg):
 //   warp 0: TMA producer for Q and K tiles; also writes each tile's count of
 //           valid key rows into a small shared ring, so that the softmax
 //           warps never read the kept lists
@@ -58,7 +57,8 @@
 //   warp 2: TMEM allocator + QK^T issuer       warp 3: PV issuer
 //   warps 4-7 and 8-11: softmax + epilogue work-groups for query columns
 //   0-31 and 32-63 (TMEM lane quarter = warp % 4)
-// Every mbarrier wait is bounded (2 s); on expiry the kernel records
+// Every mbarrier wait is bounded (2 s by default; the failure-detection entry
+// point takes another limit and can withhold one V copy); on expiry the kernel records
 // SBATTN_ERR_TIMEOUT, waits for its own copies and MMAs, frees TMEM and exits.
 #include "internal.h"
 
@@ -74,6 +74,10 @@ constexpr int kSBufs = 4;             // S^T ring in TMEM, 64 columns each
 constexpr uint32_t kColO = 256;       // four partial O^T accumulators, 64 columns each
 constexpr int kOParts = 4;
 constexpr int kInfoSlots = 16;        // per-tile valid-row counts, ring
+// registers per thread after setmaxnreg: warps 0-3 (copies, MMA issue) give
+// theirs to the softmax warps; the split must equal the launch allocation
+constexpr uint32_t kRegsIssue = 56, kRegsSoftmax = 224;
+static_assert(128 * kRegsIssue + 256 * kRegsSoftmax == kThreads * 168, "register split = 384 x 168");
 
 constexpr int kQBytes = 64 * 128 * 2;    // [2 channel halves][64 rows][128 B]
 constexpr int kKVBytes = 128 * 128 * 2;  // [2 channel halves][128 rows][128 B]
@@ -86,13 +90,10 @@ constexpr int kOffP = kOffV + kVStages * kKVBytes;
 constexpr int kOffMisc = kOffP + kPStages * kPBytes;
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// A flag raised in softmax step s (two tiles) is read in step s + kFlagDelay:
-// by then every softmax thread has finished step s (the P^T ring orders
-// them), so all read the same value without a barrier.  Slots are reused
-// every kFlagSlots steps.
-constexpr int kFlagDelay = 3;
-constexpr int kFlagSlots = 8;
-constexpr float kExpLimit = 100.0f;  // p > 2^100 is reported: sums might overflow
+// Lookahead slots: the excesses of step s are published in slot s % 4 during
+// step s - 1, read at the start of step s and cleared at the start of step
+// s + 2 (when every thread of the group has passed step s + 1's barrier).
+constexpr int kLookSlots = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Misc {
@@ -108,8 +109,9 @@ struct Misc {
   uint32_t info[kInfoSlots];  // valid key rows of a tile: low half | high half << 8
   uint32_t tmem_base;
   int abort;
-  int flag[2][kFlagSlots];  // per work-group, per softmax-step slot: a logit exceeded m by 2^8
-  uint32_t raise_req[2][32];  // per work-group: max excess per query (float bits) since the last rescale
+  uint64_t lk_bar[2];  // per work-group: the next step's excesses are published (lookahead)
+  int look_flag[2][kLookSlots];        // per work-group and step slot: some logit exceeds m by 2^8
+  uint32_t look_req[2][kLookSlots][32];  // per work-group, slot and query: largest excess (float bits)
   alignas(16) float negm2[64];  // minus the running max per query, in log2 units (read as float4)
   float alpha[64];      // rescale factors / final 1/l
   float red[2][4][32];  // cross-warp reduction scratch per work-group
@@ -193,11 +195,11 @@ SB_DEV void warp_reduce_cols(float (&v)[32], int lane) {
 // leave the others stuck.  Returns false on timeout / abort.
 struct WgSync {
   uint64_t* bar;
-  volatile int* abort;
+  WaitCtl wc;
   uint32_t phase;
   SB_DEV bool operator()() {
     mbar_arrive(bar);
-    const bool r = mbar_wait(bar, phase & 1, abort);
+    const bool r = mbar_wait(bar, phase & 1, wc);
     ++phase;
     return __all_sync(0xffffffffu, r);
   }
@@ -218,13 +220,60 @@ SB_DEV float wg_reduce_cols(float (&v)[32], float (*red)[32], int quarter, int l
   return res;
 }
 
+// A barrier of a work-group whose arrival and wait are separate points of
+// the program (bounded like every wait).
+struct SplitSync {
+  uint64_t* bar;
+  WaitCtl wc;
+  uint32_t phase;
+  SB_DEV void arrive() { mbar_arrive(bar); }
+  SB_DEV bool wait() {
+    const bool r = mbar_wait(bar, phase & 1, wc);
+    ++phase;
+    return __all_sync(0xffffffffu, r);
+  }
+};
+
+// Is key row r of a tile a real key: the tile's info word holds the valid
+// rows of its two kept blocks (low byte: rows 0-63, next byte: rows 64-127).
+SB_DEV bool key_row_valid(uint32_t info, int r, int half) {
+  return (uint32_t)(r & 63) < ((info >> (8 * half)) & 0xFFu);
+}
+
+// x <- s * c - m in the log2 domain (two lanes per instruction) for the two
+// tiles of a step; rows outside the kept set -> -inf
+SB_DEV void scale_logits(float (&x)[64], const float* negm2, float c, bool validA, bool validB) {
+  const uint64_t c2 = f2_pack(c, c);
+#pragma unroll
+  for (int q4 = 0; q4 < 8; ++q4) {
+    const float4 m4 = reinterpret_cast<const float4*>(negm2)[q4];
+    const uint64_t mlo = f2_pack(m4.x, m4.y), mhi = f2_pack(m4.z, m4.w);
+#pragma unroll
+    for (int tile = 0; tile < 2; ++tile) {
+      const int q = tile * 32 + 4 * q4;
+      const uint64_t a0 = f2_fma(f2_pack(x[q], x[q + 1]), c2, mlo);
+      const uint64_t a1 = f2_fma(f2_pack(x[q + 2], x[q + 3]), c2, mhi);
+      f2_unpack(a0, x[q], x[q + 1]);
+      f2_unpack(a1, x[q + 2], x[q + 3]);
+    }
+  }
+  if (!validA) {
+#pragma unroll
+    for (int q = 0; q < 32; ++q) x[q] = -INFINITY;
+  }
+  if (!validB) {
+#pragma unroll
+    for (int q = 0; q < 32; ++q) x[32 + q] = -INFINITY;
+  }
+}
+
 SB_DEV uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&p);
 }
 
-SB_DEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+SB_DEV bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& wc) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
 }
 
 // Walks the CTA's non-empty items and their tiles in order.
@@ -298,8 +347,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&ms->o_full, 1);
     mbar_init(&ms->o_empty, kSoftmaxThreads);
     ms->abort = 0;
-    for (int e = 0; e < 2 * kFlagSlots; ++e) (&ms->flag[0][0])[e] = 0;
-    for (int e = 0; e < 2 * 32; ++e) (&ms->raise_req[0][0])[e] = 0u;
+    mbar_init(&ms->lk_bar[0], 128);
+    mbar_init(&ms->lk_bar[1], 128);
+    for (int e = 0; e < 2 * kLookSlots; ++e) (&ms->look_flag[0][0])[e] = 0;
+    for (int e = 0; e < 2 * kLookSlots * 32; ++e) (&ms->look_req[0][0][0])[e] = 0u;
     fence_barrier_init();
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
@@ -314,7 +365,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ms->tmem_base;
   volatile int* abort_flag = &ms->abort;
+  const WaitCtl wc{abort_flag, a.wait_limit_ns};
 
+  if (warp < 4) {
+  warpgroup_regs_dec<kRegsIssue>();
   if (warp == 0 || warp == 1) {
     // ------------------------------------------------------------ producers
     const bool is_k = warp == 0;
@@ -329,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (it.ntiles == 0) continue;
       if (is_k && lane == 0) {
         const int qs = qcount % kQStages;
-        ok = mbar_wait(&ms->q_empty[qs], ((qcount / kQStages) & 1) ^ 1, abort_flag);
+        ok = mbar_wait(&ms->q_empty[qs], ((qcount / kQStages) & 1) ^ 1, wc);
         if (ok) {
           mbar_arrive_expect_tx(&ms->q_full[qs], kQBytes);
           uint8_t* dst = smem + kOffQ + qs * kQBytes;
@@ -360,8 +414,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&ms->info_full[slot]);
           }
           const int st = tcount % nstages;
-          ok = mbar_wait(&empty[st], ((tcount / nstages) & 1) ^ 1, abort_flag);
-          if (ok) {
+          if (!is_k && (int)tcount == a.withhold_v_tile) {
+            // diagnostic: this V copy is never issued (the stage is skipped),
+            // so the PV issuer's bounded wait for it must run out
+            ++tcount;
+          } else if ((ok = mbar_wait(&empty[st], ((tcount / nstages) & 1) ^ 1, wc))) {
             mbar_arrive_expect_tx(&full[st], kKVBytes);
             uint8_t* dst = smem + (is_k ? kOffK : kOffV) + st * kKVBytes;
             tma_load_4d(dst, tm, &full[st], 0, it.h, l1 * kBlock, it.b);
@@ -414,9 +471,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (is_qk) {
           const int sb = gt % kSBufs, ks = gt % kKStages, qb = ts.n % kQStages;
           const bool last = ts.t == ts.it.ntiles - 1;
-          ok = mbar_wait(&ms->s_empty[sb], ((gt / kSBufs) & 1) ^ 1, abort_flag) &&
-               mbar_wait(&ms->k_full[ks], (gt / kKStages) & 1, abort_flag) &&
-               (ts.t > 0 || mbar_wait(&ms->q_full[qb], (ts.n / kQStages) & 1, abort_flag));
+          ok = mbar_wait(&ms->s_empty[sb], ((gt / kSBufs) & 1) ^ 1, wc) &&
+               mbar_wait(&ms->k_full[ks], (gt / kKStages) & 1, wc) &&
+               (ts.t > 0 || mbar_wait(&ms->q_full[qb], (ts.n / kQStages) & 1, wc));
           if (!ok) break;
           tc_fence_after();
           const uint64_t kd = smem_desc(sbase + kOffK + ks * kKVBytes, 16, 1024, kSwizzle128B);
@@ -433,9 +490,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int vs = gt % kVStages, pb = gt % kPStages;
           const uint32_t pph = (gt / kPStages) & 1;
           const bool first = ts.t == 0, last = ts.t == ts.it.ntiles - 1;
-          ok = mbar_wait(&ms->v_full[vs], (gt / kVStages) & 1, abort_flag) &&
-               mbar_wait(&ms->p_full[pb][0], pph, abort_flag) &&
-               (!first || mbar_wait(&ms->o_empty, (ts.n & 1) ^ 1, abort_flag));
+          ok = mbar_wait(&ms->v_full[vs], (gt / kVStages) & 1, wc) &&
+               mbar_wait(&ms->p_full[pb][0], pph, wc) &&
+               (!first || mbar_wait(&ms->o_empty, (ts.n & 1) ^ 1, wc));
           if (!ok) break;
           tc_fence_after();
           // the softmax threads' P^T stores (generic proxy), acquired through
@@ -449,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < 4; ++kk)
             umma_bf16(tmem + kColO + kk * 64, vd + (uint64_t)(kk * 128), pd + (uint64_t)(kk * 128), kIdescPV, !first);
           umma_commit(&ms->p_empty[pb][0]);  // key rows 0-63 of this P^T buffer are free again
-          if (!(ok = mbar_wait(&ms->p_full[pb][1], pph, abort_flag))) break;
+          if (!(ok = mbar_wait(&ms->p_full[pb][1], pph, wc))) break;
           tc_fence_after();
           fence_proxy_async_smem();
 #pragma unroll
@@ -464,19 +521,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (!ok) {
-      if (lane == 0) {
+    if (lane == 0) {
+      if (!ok) {
         *abort_flag = 1;
         record_error(a.status, SBATTN_ERR_TIMEOUT);
-        uint64_t* drain = &ms->drain[is_qk ? 0 : 1];
-        umma_commit(drain);  // completes once every MMA this thread issued is done
-        const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < 100000000ull) {
-        }
       }
-      __syncwarp();
+      // every MMA this thread issued is done before the CTA frees TMEM, also
+      // when another role gave up first (in a normal run this wait is over at
+      // once: the softmax consumed every result)
+      uint64_t* drain = &ms->drain[is_qk ? 0 : 1];
+      umma_commit(drain);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < 100000000ull) {
+      }
     }
-  } else if (warp >= 4) {
+    __syncwarp();
+  }
+  } else {
+    warpgroup_regs_inc<kRegsSoftmax>();
     // ------------------------------------------------------ softmax + epilogue
     const int g = (warp - 4) >> 2;  // work-group: query columns [32g, 32g + 32)
     const int quarter = warp & 3;
@@ -488,10 +550,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* negm2 = ms->negm2 + col0;
     float* alpha = ms->alpha + col0;
     float(*red)[32] = ms->red[g];
-    int* flag = ms->flag[g];
-    uint32_t* raise_req = ms->raise_req[g];
+    int* look_flag = ms->look_flag[g];
+    uint32_t(*look_req)[32] = ms->look_req[g];
     uint32_t gt = 0, on = 0;  // global tile index, item ordinal
-    WgSync wg{&ms->wg_bar[g], abort_flag, 0};
+    WgSync wg{&ms->wg_bar[g], wc, 0};
+    SplitSync lk{&ms->lk_bar[g], wc, 0};
     bool ok = true;
     for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
       const Item it = decode_item(a, item);
@@ -511,14 +574,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       // The softmax takes the item's tiles two at a time (a step), so that its
       // fixed costs per wait are shared by 64 logits per thread.  S^T of a
       // step's tiles is loaded into x during the previous step (the item's
-      // first step here), hiding the TMEM load latency behind the P^T stores.
-      // Barriers signalled in tile order by one thread (S^T full, info, P^T
-      // empty) are waited on for the later tile of a step only.
+      // first step here), hiding the TMEM load latency behind the P^T stores,
+      // and is scaled and checked there too (lookahead): every thread
+      // publishes per query how far its logits of the next step exceed the
+      // running maximum, and the work-group barrier `lk` orders those
+      // publications before the next step starts.  A step whose logits run
+      // more than 2^8 above m therefore raises m first, by exactly the largest
+      // excess, before any of its p is computed: no p exceeds 2^8, whatever the
+      // scale.  Barriers signalled in tile order by one thread (S^T full, info,
+      // P^T empty) are waited on for the later tile of a step only.
+      const int nsteps = (it.ntiles + 1) >> 1;
       float x[2 * kQCols];  // [0, 32): tile A, [32, 64): tile B
+      bool validA = false, validB = false;
       {
         const bool hasB = it.ntiles > 1;
         const uint32_t gl = hasB ? gt + 1 : gt;
-        ok = warp_wait(&ms->s_full[gl % kSBufs], (gl / kSBufs) & 1, abort_flag);
+        ok = warp_wait(&ms->s_full[gl % kSBufs], (gl / kSBufs) & 1, wc);
         if (!ok) break;
         tc_fence_after();
         tmem_ld_32cols(lane_addr + (gt % kSBufs) * 64 + col0, *reinterpret_cast<uint32_t(*)[32]>(x));
@@ -526,60 +597,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_32cols(lane_addr + ((gt + 1) % kSBufs) * 64 + col0, *reinterpret_cast<uint32_t(*)[32]>(x + kQCols));
       }
 
-      for (int tA = 0; tA < it.ntiles; tA += 2) {
+      for (int step = 0; step < nsteps; ++step) {
+        const int tA = 2 * step;
         const bool hasB = tA + 1 < it.ntiles;
         const uint32_t gA = gt + tA, gB = gA + 1;
-        const uint32_t gl = hasB ? gB : gA;  // the step's last tile
-        const int step = tA >> 1;
-        if (step >= kFlagDelay && flag[(step - kFlagDelay) & (kFlagSlots - 1)]) {
-          // ---- rare path: a logit of step - kFlagDelay (or later) exceeded m
-          // by 2^8; every thread of the work-group reads the same flag, as every
-          // thread finished that step before any of them can be here.
-          if (!(ok = wg())) break;  // all threads are done with the previous step
-          if (r < kQCols) {
-            const float up = __uint_as_float(raise_req[r]);
-            alpha[r] = fast_exp2(-up);
-            negm2[r] -= up;
-            raise_req[r] = 0u;
-          }
-          if (r < kFlagSlots) flag[r] = 0;
-          if (!(ok = wg())) break;
-          // every PV issued so far must be complete before O is touched
-          const uint32_t gp = gA - 1;
-          ok = warp_wait(&ms->p_empty[gp % 2][0], (gp / 2) & 1, abort_flag) &&
-               warp_wait(&ms->p_empty[gp % 2][1], (gp / 2) & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll 1
-          for (int part = 0; part < kOParts; ++part) {
-            uint32_t o[32];
-            const uint32_t oaddr = lane_addr + kColO + part * 64 + col0;
-            tmem_ld_32cols(oaddr, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int q = 0; q < kQCols; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha[q]);
-            tmem_st_32cols(oaddr, o);
-          }
-          tmem_wait_st();
+        if (step == 0) {
+          // ---- S^T of the first step is in x: release it, seed m from it
+          tmem_wait_ld();
           tc_fence_before();
-#pragma unroll
-          for (int q = 0; q < kQCols; q += 2) l2[q >> 1] = f2_mul(l2[q >> 1], f2_pack(alpha[q], alpha[q + 1]));
-        }
-        // ---- S^T of the step's tiles (this work-group's 32 query columns) is in x
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&ms->s_empty[gA % kSBufs]);
-        if (hasB) mbar_arrive(&ms->s_empty[gB % kSBufs]);
-        // ---- are my key rows real keys (counts written by the K producer)
-        ok = warp_wait(&ms->info_full[gl % kInfoSlots], (gl / kInfoSlots) & 1, abort_flag);
-        if (!ok) break;
-        const uint32_t infoA = ms->info[gA % kInfoSlots];
-        const uint32_t infoB = hasB ? ms->info[gB % kInfoSlots] : 0u;
-        const bool validA = (uint32_t)(r & 63) < ((infoA >> (8 * half)) & 0xFFu);
-        const bool validB = (uint32_t)(r & 63) < ((infoB >> (8 * half)) & 0xFFu);
-
-        if (tA == 0) {
-          // seed the running max from the first step
+          mbar_arrive(&ms->s_empty[gA % kSBufs]);
+          if (hasB) mbar_arrive(&ms->s_empty[gB % kSBufs]);
+          const uint32_t gl = hasB ? gB : gA;
+          ok = warp_wait(&ms->info_full[gl % kInfoSlots], (gl / kInfoSlots) & 1, wc);
+          if (!ok) break;
+          validA = key_row_valid(ms->info[gA % kInfoSlots], r, half);
+          validB = hasB && key_row_valid(ms->info[gB % kInfoSlots], r, half);
           float v[kQCols];
 #pragma unroll
           for (int q = 0; q < kQCols; ++q)
@@ -588,48 +620,54 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           if (r < kQCols) negm2[r] = (mx == -INFINITY) ? 0.f : -mx;
           if (!(ok = wg())) break;
-        }
-        // ---- x <- s * c - m (log2 domain), two lanes per instruction; rows
-        // outside the kept set -> -inf
-        float lmax = -INFINITY;
-        {
-          const uint64_t c2 = f2_pack(c, c);
-#pragma unroll
-          for (int q4 = 0; q4 < kQCols / 4; ++q4) {
-            const float4 m4 = reinterpret_cast<const float4*>(negm2)[q4];
-            const uint64_t mlo = f2_pack(m4.x, m4.y), mhi = f2_pack(m4.z, m4.w);
-#pragma unroll
-            for (int tile = 0; tile < 2; ++tile) {
-              const int q = tile * kQCols + 4 * q4;
-              const uint64_t a0 = f2_fma(f2_pack(x[q], x[q + 1]), c2, mlo);
-              const uint64_t a1 = f2_fma(f2_pack(x[q + 2], x[q + 3]), c2, mhi);
-              f2_unpack(a0, x[q], x[q + 1]);
-              f2_unpack(a1, x[q + 2], x[q + 3]);
+          scale_logits(x, negm2, c, validA, validB);
+        } else {
+          // ---- every thread of the group has published this step's excess
+          if (!(ok = lk.wait())) break;
+          const int sl = step & (kLookSlots - 1);
+          if (look_flag[sl]) {
+            // ---- rare path: some logit of this step exceeds m by more than
+            // 2^8: raise m by the largest excess of each query, now
+            if (r < kQCols) {
+              const float up = __uint_as_float(look_req[sl][r]);
+              alpha[r] = fast_exp2(-up);
+              negm2[r] -= up;
             }
-          }
-          if (!validA) {
+            if (!(ok = wg())) break;  // the new m is visible to the group
 #pragma unroll
-            for (int q = 0; q < kQCols; ++q) x[q] = -INFINITY;
-          }
-          if (!validB) {
+            for (int q = 0; q < kQCols; ++q) {
+              const float up = __uint_as_float(look_req[sl][q]);
+              x[q] -= up;
+              x[kQCols + q] -= up;
+            }
+            // every PV issued so far must be complete before O is touched
+            const uint32_t gp = gA - 1;
+            ok = warp_wait(&ms->p_empty[gp % 2][0], (gp / 2) & 1, wc) &&
+                 warp_wait(&ms->p_empty[gp % 2][1], (gp / 2) & 1, wc);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int part = 0; part < kOParts; ++part) {
+              uint32_t o[32];
+              const uint32_t oaddr = lane_addr + kColO + part * 64 + col0;
+              tmem_ld_32cols(oaddr, o);
+              tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < kQCols; ++q) x[kQCols + q] = -INFINITY;
-          }
+              for (int q = 0; q < kQCols; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha[q]);
+              tmem_st_32cols(oaddr, o);
+            }
+            tmem_wait_st();
+            tc_fence_before();
 #pragma unroll
-          for (int q = 0; q < kQCols; q += 2)
-            lmax = fmax3(lmax, fmaxf(x[q], x[q + 1]), fmaxf(x[kQCols + q], x[kQCols + q + 1]));
-        }
-        if (lmax > kRescaleThreshold) {
-          // rare: ask a later step to raise m for these queries (logits are
-          // exact meanwhile up to 2^100 above m; beyond that the call reports
-          // a device error)
-#pragma unroll
-          for (int q = 0; q < kQCols; ++q) {
-            const float ex = fmaxf(x[q], x[kQCols + q]);
-            if (ex > kRescaleThreshold) atomicMax(&raise_req[q], __float_as_uint(ex));
+            for (int q = 0; q < kQCols; q += 2) l2[q >> 1] = f2_mul(l2[q >> 1], f2_pack(alpha[q], alpha[q + 1]));
           }
-          flag[step & (kFlagSlots - 1)] = 1;
-          if (lmax > kExpLimit) record_error(a.status, SBATTN_ERR_DEVICE);
+          // the slot of two steps ago is read by every thread of the group
+          // (they all passed this step's lk) and is next written two steps on
+          if (step >= 2) {
+            const int old = (step - 2) & (kLookSlots - 1);
+            if (r < kQCols) look_req[old][r] = 0u;
+            if (r == 0) look_flag[old] = 0;
+          }
         }
         // ---- p = 2^x and partial row sums (a row outside the kept set has
         // x = -inf and p = 0); the row sums take the bf16 weights PV actually
@@ -647,10 +685,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         // ---- start loading the next step's S^T
-        if (tA + 2 < it.ntiles) {
-          const bool nB = tA + 3 < it.ntiles;
-          const uint32_t gn = gA + 2, gnl = nB ? gn + 1 : gn;
-          ok = warp_wait(&ms->s_full[gnl % kSBufs], (gnl / kSBufs) & 1, abort_flag);
+        const bool more = step + 1 < nsteps;
+        const bool nB = tA + 3 < it.ntiles;
+        const uint32_t gn = gA + 2;
+        if (more) {
+          const uint32_t gnl = nB ? gn + 1 : gn;
+          ok = warp_wait(&ms->s_full[gnl % kSBufs], (gnl / kSBufs) & 1, wc);
           if (!ok) break;
           tc_fence_after();
           tmem_ld_32cols(lane_addr + (gn % kSBufs) * 64 + col0, *reinterpret_cast<uint32_t(*)[32]>(x));
@@ -665,7 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (tile == 1 && !hasB) break;
           const uint32_t gx = gA + tile;
           const int pb = gx % 2;
-          ok = warp_wait(&ms->p_empty[pb][half], ((gx / 2) & 1) ^ 1, abort_flag);
+          ok = warp_wait(&ms->p_empty[pb][half], ((gx / 2) & 1) ^ 1, wc);
           if (!ok) break;
           uint8_t* prow = smem + kOffP + pb * kPBytes + r * 128;
 #pragma unroll
@@ -679,12 +719,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         // instead of one per softmax thread and step here)
         mbar_arrive(&ms->p_full[gA % 2][half]);
         if (hasB) mbar_arrive(&ms->p_full[gB % 2][half]);
+        // ---- lookahead: scale the next step's logits and publish how far
+        // they exceed the running maximum
+        if (more) {
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(&ms->s_empty[gn % kSBufs]);
+          if (nB) mbar_arrive(&ms->s_empty[(gn + 1) % kSBufs]);
+          const uint32_t gnl = nB ? gn + 1 : gn;
+          ok = warp_wait(&ms->info_full[gnl % kInfoSlots], (gnl / kInfoSlots) & 1, wc);
+          if (!ok) break;
+          validA = key_row_valid(ms->info[gn % kInfoSlots], r, half);
+          validB = nB && key_row_valid(ms->info[(gn + 1) % kInfoSlots], r, half);
+          scale_logits(x, negm2, c, validA, validB);
+          float lmax = -INFINITY;
+#pragma unroll
+          for (int q = 0; q < 2 * kQCols; q += 2) lmax = fmax3(lmax, x[q], x[q + 1]);
+          if (lmax > kRescaleThreshold) {
+            const int sl = (step + 1) & (kLookSlots - 1);
+#pragma unroll
+            for (int q = 0; q < kQCols; ++q) {
+              const float ex = fmaxf(x[q], x[kQCols + q]);
+              if (ex > kRescaleThreshold) atomicMax(&look_req[sl][q], __float_as_uint(ex));
+            }
+            look_flag[sl] = 1;
+          }
+          lk.arrive();
+        }
       }
       if (!ok) break;
       gt += it.ntiles;
 
       // ---- epilogue: (sum of the partial O^T) / l -> out ----
-      ok = warp_wait(&ms->o_full, on & 1, abort_flag);
+      ok = warp_wait(&ms->o_full, on & 1, wc);
       if (!ok) break;
       tc_fence_after();
       {
@@ -697,9 +764,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         if (r < kQCols) {
           alpha[r] = lsum > 0.f ? 1.0f / lsum : 0.f;
-          raise_req[r] = 0u;
+#pragma unroll
+          for (int sl = 0; sl < kLookSlots; ++sl) look_req[sl][r] = 0u;
         }
-        if (r < kFlagSlots) flag[r] = 0;
+        if (r < kLookSlots) look_flag[r] = 0;
         if (!(ok = wg())) break;
       }
       float acc[kQCols];
@@ -758,6 +826,11 @@ int launch_attention(const AttentionArgs& a, cudaStream_t stream) {
   if (cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
       cudaSuccess)
     return SBATTN_ERR_CUDA;
+  // setmaxnreg moves registers between warpgroups within the CTA's launch
+  // allocation; the split (kRegsIssue / kRegsSoftmax) adds up to exactly
+  // 384 x 168, so the kernel must be built with 168 registers per thread
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, attention_kernel) != cudaSuccess || fa.numRegs != 168) return SBATTN_ERR_CUDA;
   const long total = (long)a.B * a.H * a.nblk;
   const int grid = (int)(total < sms ? total : sms);
   attention_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps[0], maps[1], maps[2], a);

@@ -86,18 +86,23 @@ SB_DEV bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns
   return done != 0;
 }
 
-// Wait for the phase of `bar` with the given parity to complete.  Bounded:
-// gives up after kWaitLimitNs of wall time, or as soon as *abort becomes
-// nonzero (another role gave up), and returns false in both cases.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+// Limits of a bounded wait: give up once *abort becomes nonzero (another
+// role gave up) or after limit_ns of wall time.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s, the default limit
+struct WaitCtl {
+  volatile int* abort;
+  uint64_t limit_ns;
+};
 
-SB_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// Wait for the phase of `bar` with the given parity to complete.  Bounded by
+// `w`; returns false when it gives up.
+SB_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
-    if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if (*w.abort) return false;
+    if (global_timer_ns() - t0 > w.limit_ns) return false;
   }
 }
 

@@ -78,6 +78,8 @@ struct AttentionArgs {
   int32_t* status;
   int B, N, H, nblk, K_capacity;
   float scale;
+  unsigned long long wait_limit_ns;  // limit of every bounded wait inside the kernel
+  int withhold_v_tile;               // diagnostic: per-CTA V tile never copied (-1: none)
 };
 
 int launch_attention(const AttentionArgs& a, cudaStream_t stream);

@@ -225,18 +225,39 @@ SBATTN_API int sbattn_select_blocks_noalloc(const uint16_t* q_rot, const uint16_
  *   status          optional device int32 (may be NULL).  If given, the
  *                   kernel stores a nonzero SBATTN_ERR_* code there when a
  *                   kept index or count is out of range (that block/row is
- *                   skipped; DEVICE), when a logit exceeds the row's running
- *                   maximum by more than 100 in log2 units before the
- *                   maximum is raised (its weight 2^x could overflow the
- *                   sums; DEVICE), or when a bounded internal wait runs out
- *                   (TIMEOUT); it never clears it.  Zero it before the call and read it after the
- *                   stream has reached the call.
+ *                   skipped; DEVICE) or when a bounded internal wait runs out
+ *                   (TIMEOUT); it never clears it.  Zero it before the call
+ *                   and read it after the stream has reached the call (e.g.
+ *                   with sbattn_check_status).
+ * The softmax is exact for any logit range: the running maximum of a query
+ * is raised before any weight of a step is computed whenever the step's
+ * logits exceed it by more than 2^8 (so every weight is at most 2^8).
  * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (d != 128), MISALIGNED, CUDA.
  */
 SBATTN_API int sbattn_forward(const uint16_t* q_rot, const uint16_t* k_rot, const uint16_t* v,
                               const int32_t* kept_idx, const int32_t* kept_cnt, int K_capacity,
                               uint16_t* out, int B, int N, int H, int d,
                               float softmax_scale, int32_t* status, void* stream);
+
+/* Failure-detection form of sbattn_forward (the pages have no counterpart;
+ * it exists so that tests can show that the kernel's internal waits are
+ * bounded).  Same computation and arguments, plus:
+ *   wait_limit_ns    limit of every bounded wait inside the kernel, in
+ *                    [1 ms, 20 s] (sbattn_forward uses 2 s)
+ *   withhold_v_tile  -1 for a normal call; t >= 0 makes every CTA skip the
+ *                    copy of its t-th V tile (counted in the CTA's own order
+ *                    of kept-block pairs), so the wait for that tile runs out:
+ *                    the kernel then stores SBATTN_ERR_TIMEOUT in `status`,
+ *                    lets its own copies and matrix products finish, frees
+ *                    its tensor memory and returns; the outputs of the call
+ *                    are undefined, the device stays usable.
+ * Errors: as sbattn_forward; INVALID_ARG for a limit or tile out of range.
+ */
+SBATTN_API int sbattn_forward_diag(const uint16_t* q_rot, const uint16_t* k_rot, const uint16_t* v,
+                                   const int32_t* kept_idx, const int32_t* kept_cnt, int K_capacity,
+                                   uint16_t* out, int B, int N, int H, int d, float softmax_scale,
+                                   int32_t* status, unsigned long long wait_limit_ns, int withhold_v_tile,
+                                   void* stream);
 
 /* ---- 4. fused DiT-block elementwise steps around attention -------------
  * [p3] "先把近两倍的免费收益拿走": the lossless gain also comes from fused

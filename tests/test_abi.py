@@ -163,6 +163,17 @@ def test_forward_validation(L):
     assert _forward(L, B=1 << 20, N=1 << 20, H=1 << 10) == SHAPE  # item count overflows int32
 
 
+def test_forward_diag_validation(L):
+    """The failure-detection form: its limit and withheld tile are checked on
+    the host before anything else (no GPU needed)."""
+    args = (A, A + 0x100000, A + 0x200000, A + 0x300000, A + 0x400000, 4, A + 0x500000, 1, 256, 2, 128, 0.0, None)
+    assert L.sbattn_forward_diag(*args, 999_999, -1, None) == INVALID          # limit below 1 ms
+    assert L.sbattn_forward_diag(*args, 20_000_000_001, -1, None) == INVALID   # above 20 s
+    assert L.sbattn_forward_diag(*args, 50_000_000, -2, None) == INVALID
+    bad = (A, A + 0x100000, None) + args[3:]
+    assert L.sbattn_forward_diag(*bad, 50_000_000, 0, None) == INVALID       # then the usual checks
+
+
 def _adaln(L, x=A, shift=A + 0x1000, scale=A + 0x2000, out=A + 0x100000, B=2, N=300, C=5120, eps=1e-6):
     return L.sbattn_adaln_modulate(x, shift, scale, out, B, N, C, eps, None)
 
