@@ -98,3 +98,24 @@ def test_full_size_sampled(name):
 
     stats = _chain_compare(wl, _View, x_cpu, out_cpu, range(len(heads)), 12, rng)
     assert stats["rows"] >= 2 * 12
+
+
+def test_host_buffer_calls_are_pipelined_and_equal_the_device_path():
+    """Back-to-back calls with host (pinned) tensors reuse two device slots,
+    with the copies on their own streams; every call's output must equal
+    the device path's on the same inputs, bit for bit."""
+    wl = custom_workload("pipe", B=1, H=4, T=3, Hh=16, W=40, sparsity=0.6, seed=51)
+    inputs = [make_inputs(wl, seed=s) for s in (51, 52, 53, 54, 55)]
+    layer = sb.AttentionLayer(wl.B, wl.T, wl.Hh, wl.W, wl.H, wl.sparsity, device=DEV)
+    outs = []
+    for x in inputs:
+        host = {k: v.pin_memory() for k, v in x.items()}
+        outs.append(layer(host["q"], host["k"], host["v"], host["w_q"], host["w_k"]))
+    layer.drain()
+    torch.cuda.synchronize()
+    layer.check_status()
+    ref_layer = sb.AttentionLayer(wl.B, wl.T, wl.Hh, wl.W, wl.H, wl.sparsity, device=DEV)
+    for x, got in zip(inputs, outs):
+        d = {k: v.to(DEV) for k, v in x.items()}
+        ref = ref_layer.run_device(d["q"], d["k"], d["v"], d["w_q"], d["w_k"]).cpu()
+        assert torch.equal(got, ref)
