@@ -6,69 +6,99 @@
 // skipped).
 //
 // Scores on tensor cores.  A work item is 128 query blocks of one (batch,
-// head), one per TMEM lane, so that a thread owns a query block's whole score
-// row and selects within it alone.  The block scores s_ij = q_bar_i . k_bar_j
-// are fp32 dot products; the tensor core computes them from tf32 pieces:
-// x = hi + lo with hi = x with its low 13 mantissa bits cleared (exactly a
-// tf32 value) and lo = x - hi, and s = hi_q.hi_k + hi_q.lo_k + lo_q.hi_k
-// (kind::tf32, fp32 accumulation; the dropped lo.lo term and the tf32
-// reading of lo leave an error of a few 1e-6 of |q_bar_i| |k_bar_j|).
-//   * Q pieces: each selector thread loads its query block's mean, splits it
-//     and stores hi / lo into its own TMEM lane (the A operand, read from
-//     tensor memory).
+// head), one per TMEM lane.  The block scores s_ij = q_bar_i . k_bar_j are
+// fp32 dot products; the tensor core computes them from tf32 pieces: x = hi +
+// lo with hi = x with its low 13 mantissa bits cleared (exactly a tf32 value)
+// and lo = x - hi, and s = hi_q.hi_k + hi_q.lo_k + lo_q.hi_k (kind::tf32, fp32
+// accumulation; the dropped lo.lo term and the tf32 reading of lo leave an
+// error of a few 1e-6 of |q_bar_i| |k_bar_j|).  A pass over the row streams
+// the key blocks in tiles of 128: M = 128 query blocks, N = 128 key blocks,
+// K = 8 channels per MMA, 16 K-steps x 3 products per tile into one of two
+// accumulators of 128 TMEM columns, so that the tensor core fills one while
+// the other is read.  The same inputs and instruction sequence give the same
+// scores in every pass.
+//   * Q pieces: the selector threads load their query block's mean (each of
+//     the two selector warpgroups half of the channels), split it and store
+//     hi / lo into the block's TMEM lane (the A operand).
 //   * K pieces: a TMA warp streams k_bar in stages of 128 key blocks x 32
 //     channels (one 128-byte swizzle row of fp32 per key block), four stages
 //     deep; four converter warps split each stage in place into hi (where TMA
 //     wrote it) and lo (a second buffer with the same swizzled positions).
-//   * One thread issues the MMAs: per channel chunk of a group of 256 key
-//     blocks (two stages) 4 K-steps x 3 products x 2 tiles, M = 128 query
-//     blocks, N = 128 keys, K = 8 channels, into two accumulators of 128 TMEM
-//     columns (the two tiles' chains interleave).
-// Exact top-K: an 8-bit radix select on order-preserving 32-bit keys of the
-// fp32 scores, four passes (most significant digit first), each counting in a
-// per-row histogram (u16, shared memory) the digits of the keys that match
-// the digits found so far; then an output pass writes, in ascending key
-// block order, the diagonal, every score above the selected value and the
-// lowest-indexed ties.  The scores are recomputed by the tensor core in every
-// pass: deterministic, so all passes see the same values.  Threshold mode
-// (keep s >= tau) and the trivial budgets need the output pass only.
+//   * The tiles of a pass alternate between the two selector warpgroups: the
+//     first takes tiles 0, 1, 2, ... (accumulator 0), the second tiles T-1,
+//     T-2, ... (accumulator 1), so that each writes its kept blocks in order
+//     from its own end of the output row.
+// Exact top-K per row, in four passes over the scores:
+//   1. sample: one tile of every ceil(nblk/128)-th key block, one product
+//      (hi.hi); mean m and deviation sd of the row's sampled scores place a
+//      window of 2 sd around m + z sd, z the normal quantile of the kept
+//      fraction;
+//   2. histogram: 256 bins, 254 across the window and one for each side,
+//      bin(s) = round(clamp(s * A + B, 0, 255)), a non-decreasing function of
+//      s; the bin holding the (K-1)-th largest off-diagonal score follows from
+//      the counts (u16 per row in shared memory, fire-and-forget atomics);
+//   3. compaction: the scores of that bin (a few dozen at most) go to
+//      shared memory with their block index; the (K-1)-th largest under the
+//      order (score descending, block index ascending) among them is the cut;
+//   4. output: the diagonal and every block at or above the cut, in
+//      ascending block order.
+// If some row's bin holds more than 32 blocks (a sample that misplaced the
+// window, or mass ties), the item runs instead six radix levels restricted to
+// that bin: the four bytes of an order-preserving key of the score, then the
+// two bytes of (65535 - block index), which fixes the cut exactly.  Threshold
+// mode (keep s >= tau) and the trivial budgets run the output pass alone.
 //
-// Roles (384 threads, one CTA per SM, persistent over work items):
+// Roles (512 threads, one CTA per SM, persistent over work items):
 //   warp 0: TMA producer           warp 1: TMEM allocator + MMA issuer
-//   warps 4-7: converters          warps 8-11: selectors (TMEM lane quarter = warp % 4)
-// Every mbarrier wait is bounded; on expiry the kernel stores nothing more,
-// lets its own copies and MMAs finish, frees TMEM and returns.
+//   warps 4-7: converters          warps 8-15: two selector warpgroups
+//                                  (TMEM lane quarter = warp % 4)
+// Every mbarrier wait is bounded; a failed wait is shared with the other
+// selector warpgroup at the next named barrier, after which the kernel stores
+// nothing more, lets its own copies and MMAs finish, frees TMEM and returns.
 #include "internal.h"
 
 namespace sbattn {
 
 namespace {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
 constexpr int kRows = 128;                    // query blocks per work item (MMA M)
-constexpr int kTileN = 128;                   // key blocks per MMA (N)
-constexpr int kGroupTiles = 2;                // accumulators per group
-constexpr int kGroupKeys = kTileN * kGroupTiles;      // 256
+constexpr int kTileN = 128;                   // key blocks per tile (MMA N)
 constexpr int kChunkD = 32;                   // channels per stage (128 bytes of fp32)
 constexpr int kChunks = kHeadDim / kChunkD;   // 4
-constexpr int kStages = 4;                    // a stage: one tile of 128 keys x one chunk of 32 channels
+constexpr int kStages = 4;                    // a stage: one tile x one chunk of 32 channels
 constexpr int kHalfBytes = kTileN * kChunkD * 4;      // 16 KB: hi (TMA target) or lo
 constexpr int kStageBytes = 2 * kHalfBytes;
 constexpr int kBins = 256;
 constexpr int kHistBytes = kBins * kRows * 2;         // u16 counts, [bin][row]
 constexpr int kOffHist = kStages * kStageBytes;       // 128 KB
+constexpr int kCap = 32;                              // candidates per row and selector warpgroup
+// candidates reuse the (then zero) histogram space: f32 scores [wg][slot][row],
+// then u16 block indices [wg][slot][row]
+constexpr int kOffCandJ = kOffHist + 2 * kCap * kRows * 4;
+static_assert(kOffCandJ + 2 * kCap * kRows * 2 <= kOffHist + kHistBytes, "candidates fit the histogram space");
 constexpr int kOffMisc = kOffHist + kHistBytes;       // 192 KB
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColQhi = 0, kColQlo = 128, kColD = 256;
-constexpr int kRadixPasses = 4;
+constexpr uint32_t kColQhi = 0, kColQlo = 128, kColD = 256;  // accumulator b at kColD + 128 b
+constexpr int kLevels = 6;                    // fallback: 4 key bytes + 2 index bytes
+constexpr float kWindowSd = 1.0f;             // half-width of the histogram window, in sd
+
+enum PassKind { kSample = 0, kHist = 1, kCompact = 2, kLevel = 3, kOutput = 4 };
 
 struct Misc {
   uint64_t raw_full[kStages], conv_full[kStages], stage_empty[kStages];
-  uint64_t d_full, d_empty;  // the group's accumulators
-  uint64_t q_ready, q_empty;  // the item's Q pieces in TMEM
+  uint64_t d_full[2], d_empty[2];  // accumulator b belongs to selector warpgroup b
+  uint64_t q_ready, q_empty;       // the item's Q pieces in TMEM
+  uint64_t plan;                   // one phase per item: fast or fallback schedule
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  int plan_slow;
+  // per query block of the item, written by the first selector warpgroup
+  float bin_a[kRows], bin_b[kRows], cut_s[kRows];
+  int cut_j[kRows], tb[kRows];
+  uint32_t kpre[kRows], kmask[kRows], vpre[kRows], vmask[kRows];
+  int n1[kRows], w0[kRows], w1[kRows];
 };
 constexpr int kSmemBytes = kOffMisc + (int)sizeof(Misc);
 
@@ -94,31 +124,220 @@ SB_DEV void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0
       : "memory");
 }
 
+// Named barriers of the 256 selector threads: a plain one, and reductions of
+// a predicate over all of them.
+SB_DEV void sel_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+SB_DEV bool sel_and(bool p) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred a, b;\n\tsetp.ne.u32 a, %1, 0;\n\tbar.red.and.pred b, 2, 256, a;\n\t"
+      "selp.u32 %0, 1, 0, b;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)p)
+      : "memory");
+  return r != 0;
+}
+SB_DEV bool sel_or(bool p) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred a, b;\n\tsetp.ne.u32 a, %1, 0;\n\tbar.red.or.pred b, 3, 256, a;\n\t"
+      "selp.u32 %0, 1, 0, b;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)p)
+      : "memory");
+  return r != 0;
+}
+
 // Monotone map from float to uint32 (larger float -> larger key); adding
 // +0 first turns -0 into +0, so that the two zeros are equal keys.
 SB_DEV uint32_t order_key(float f) {
   const uint32_t u = __float_as_uint(f + 0.0f);
   return u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
 }
+SB_DEV float key_value(uint32_t k) { return __uint_as_float((k & 0x80000000u) ? (k ^ 0x80000000u) : ~k); }
+
+// Histogram bin of a score: round(clamp(s * A + B, 0, 255)).  Each step is
+// non-decreasing in s (fma, min, max, and rounding to an integer by adding
+// 1.5 * 2^23), so a higher bin means a strictly higher score.
+SB_DEV uint32_t bin_of(float s, float A, float B) {
+  const float x = fminf(fmaxf(fmaf(s, A, B), 0.0f), 255.0f);
+  return __float_as_uint(x + 12582912.0f) & 0xFFu;
+}
 
 SB_DEV uint32_t tf32_hi(uint32_t u) { return u & 0xFFFFE000u; }
 
 // The schedule every role walks: work items (128 query blocks of one
-// batch-head) strided over the grid, passes, groups of 256 key blocks and the
-// four channel chunks of a group.
+// batch-head) strided over the grid, passes, the tiles of a pass (in the
+// order tile_of gives) and the four channel chunks of a tile.
 struct Plan {
-  int items, row_blocks, groups, passes;
+  int items, row_blocks, tiles, stride, ns;
+  bool general;  // budget form with 1 < keep < nblk
   SB_DEV void init(const SelectArgs& a) {
     row_blocks = (a.nblk + kRows - 1) / kRows;
     items = a.B * a.H * row_blocks;
-    groups = (a.nblk + kGroupKeys - 1) / kGroupKeys;
-    const bool radix = !a.threshold_mode && a.keep > 1 && a.keep < a.nblk;
-    passes = radix ? kRadixPasses + 1 : 1;
+    tiles = (a.nblk + kTileN - 1) / kTileN;
+    stride = (a.nblk + kTileN - 1) / kTileN;  // sampled blocks: j = m * stride, m < ns <= 128
+    ns = (a.nblk + stride - 1) / stride;
+    general = !a.threshold_mode && a.keep > 1 && a.keep < a.nblk;
   }
+  SB_DEV int total(bool slow) const { return general ? (slow ? 3 + kLevels : 4) : 1; }
+  SB_DEV int kind(int p, bool slow) const {
+    if (!general) return kOutput;
+    if (p == 0) return kSample;
+    if (p == 1) return kHist;
+    if (!slow) return p == 2 ? kCompact : kOutput;
+    return p < 2 + kLevels ? kLevel : kOutput;
+  }
+  SB_DEV int ntiles(int kind) const { return kind == kSample ? 1 : tiles; }
+};
+// Position pos of a pass -> tile: even positions ascend from tile 0, odd ones
+// descend from the last tile.
+SB_DEV int tile_of(int pos, int tiles) { return (pos & 1) ? tiles - 1 - (pos >> 1) : (pos >> 1); }
+
+// What one selector thread carries through a tile.
+struct Row {
+  int i, nblk;              // my query block, key blocks
+  bool row;                 // i < nblk
+  float A, B;               // histogram bin map
+  uint32_t tb;              // the bin being resolved
+  float cs;                 // cut: keep s > cs, or s == cs and j <= cj
+  int cj;
+  uint32_t kpre, kmask, vpre, vmask, sh;  // fallback radix state
+  bool vlevel;              // fallback level on the block index bytes
+  uint32_t* hw;             // my 16-bit histogram lane: + bin * 64 words
+  uint32_t inc;
+  float* cand_s;            // my candidate slots: + slot * kRows
+  uint16_t* cand_j;
+  int n;                    // candidates found
+  int32_t* out;             // my output row
+  int w, top;               // kept blocks written; first position of the second warpgroup
+  bool desc;                // second warpgroup: writes backwards from top
+  int cap;
+  float* srow;              // scores dump row or null
+  float sum, sq;            // sampled scores
+  int ns_seen;
+  int stride, ns;
 };
 
+// Output decision for block j with score bits u: the diagonal and every block
+// at or above the cut are written, in my direction.
+SB_DEV void output_one(uint32_t u, int j, bool checks, Row& R) {
+  if (checks && j >= R.nblk) return;
+  const float s = __uint_as_float(u);
+  if (R.srow != nullptr) R.srow[j] = s;
+  const bool kept = (checks && j == R.i) || s > R.cs || (s == R.cs && j <= R.cj);
+  if (kept) {
+    const int pos = R.desc ? R.top - R.w : R.w;
+    if (pos >= 0 && pos < R.cap) R.out[pos] = j;  // bounded by the row's capacity
+    ++R.w;
+  }
+}
+
+// One chunk of 32 scores of my row, block indices j0 .. j0+31 (sample pass:
+// sample indices m0 .. m0+31).  `checks`: the tile holds the diagonal or runs
+// past nblk (or is the sample), so each element is tested.
+template <int Kind>
+SB_DEV void scan_chunk(const uint32_t (&v)[32], int j0, bool checks, Row& R) {
+  if (Kind == kSample) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int m = j0 + e, j = m * R.stride;
+      const float s = __uint_as_float(v[e]);
+      if (m < R.ns && j != R.i) {
+        R.sum += s;
+        R.sq = fmaf(s, s, R.sq);
+        ++R.ns_seen;
+      }
+    }
+  } else if (Kind == kHist) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int j = j0 + e;
+      const uint32_t b = bin_of(__uint_as_float(v[e]), R.A, R.B);
+      if (!checks || (j < R.nblk && j != R.i)) atomicAdd(R.hw + b * 64u, R.inc);
+    }
+  } else if (Kind == kCompact) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int j = j0 + e;
+      const float s = __uint_as_float(v[e]);
+      if (bin_of(s, R.A, R.B) == R.tb && (!checks || (j < R.nblk && j != R.i))) {
+        if (R.n < kCap) {
+          R.cand_s[R.n * kRows] = s;
+          R.cand_j[R.n * kRows] = (uint16_t)j;
+        }
+        ++R.n;
+      }
+    }
+  } else if (Kind == kLevel) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int j = j0 + e;
+      const float s = __uint_as_float(v[e]);
+      const uint32_t key = order_key(s), vj = 0xFFFFu - (uint32_t)j;
+      const bool member = bin_of(s, R.A, R.B) == R.tb && (key & R.kmask) == R.kpre && (vj & R.vmask) == R.vpre;
+      const uint32_t digit = ((R.vlevel ? vj : key) >> R.sh) & 0xFFu;
+      if (member && (!checks || (j < R.nblk && j != R.i))) atomicAdd(R.hw + digit * 64u, R.inc);
+    }
+  } else {  // kOutput, in my writing direction (constant register indices either way)
+    if (R.desc) {
+#pragma unroll
+      for (int e = 31; e >= 0; --e) output_one(v[e], j0 + e, checks, R);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) output_one(v[e], j0 + e, checks, R);
+    }
+  }
+}
+
+// My 128 columns of accumulator `d` (lane quarter address), in four chunks of
+// 32 with the next chunk's load in flight; descending chunk order for the
+// backward writer.
+template <int Kind>
+SB_DEV void scan_tile(uint32_t d, int jbase, bool checks, Row& R) {
+  uint32_t va[32], vb[32];
+  const bool back = Kind == kOutput && R.desc;
+  tmem_ld_32cols(d + (back ? 96u : 0u), va);
+#pragma unroll 1
+  for (int h = 0; h < 2; ++h) {
+    const int ca = back ? 3 - 2 * h : 2 * h, cb = back ? 2 - 2 * h : 2 * h + 1;
+    tmem_wait_ld_regs(va);
+    tmem_ld_32cols(d + (uint32_t)cb * 32u, vb);
+    if (R.row) scan_chunk<Kind>(va, jbase + ca * 32, checks, R);
+    tmem_wait_ld_regs(vb);
+    if (h == 0) tmem_ld_32cols(d + (back ? 32u : 64u), va);
+    if (R.row) scan_chunk<Kind>(vb, jbase + cb * 32, checks, R);
+  }
+}
+
+// Scan my row's 256 bins from the top (clearing them) for the bin where the
+// running count reaches `need`; returns it (or -1) with the count above it
+// and its own count.
+SB_DEV int find_bin(const uint16_t* hist_row, int need, int& above, int& cnt) {
+  uint16_t* h = const_cast<uint16_t*>(hist_row);
+  int cum = 0, bin = -1;
+  above = 0;
+  cnt = 0;
+#pragma unroll 4
+  for (int b = kBins - 1; b >= 0; --b) {
+    const int c = h[b * kRows];
+    h[b * kRows] = 0;
+    if (bin < 0) {
+      if (cum + c >= need) {
+        bin = b;
+        above = cum;
+        cnt = c;
+      } else {
+        cum += c;
+      }
+    }
+  }
+  return bin;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-    select_kernel(const __grid_constant__ CUtensorMap tm_k, SelectArgs a, uint64_t wait_limit_ns) {
+    select_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_s, SelectArgs a,
+                  uint64_t wait_limit_ns) {
   extern __shared__ __align__(1024) uint8_t smem[];
   Misc* ms = reinterpret_cast<Misc*>(smem + kOffMisc);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -132,20 +351,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ms->conv_full[s], 128);
       mbar_init(&ms->stage_empty[s], 1);
     }
-    mbar_init(&ms->d_full, 1);
-    mbar_init(&ms->d_empty, 128);
-    mbar_init(&ms->q_ready, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ms->d_full[b], 1);
+      mbar_init(&ms->d_empty[b], 128);
+    }
+    mbar_init(&ms->q_ready, 256);
     mbar_init(&ms->q_empty, 1);
+    mbar_init(&ms->plan, 1);
     mbar_init(&ms->drain, 1);
     ms->abort = 0;
+    ms->plan_slow = 0;
     fence_barrier_init();
     prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_s);
   }
   if (warp == 1) {
     tmem_alloc(&ms->tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  // histograms start at zero; every radix pass clears the bins it read
+  // histograms start at zero; every level clears the bins it read and the
+  // compaction clears the candidate slots it used
   for (int e = threadIdx.x; e < kHistBytes / 16; e += kThreads)
     reinterpret_cast<uint4*>(smem + kOffHist)[e] = make_uint4(0u, 0u, 0u, 0u);
   tc_fence_before();
@@ -153,26 +378,39 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ms->tmem_base;
   volatile int* abort_flag = &ms->abort;
+  volatile int* plan_slow = &ms->plan_slow;
   const WaitCtl wc{abort_flag, wait_limit_ns};
 
   if (warp == 0) {
     // ------------------------------------------------------------- TMA
     bool ok = true;
-    uint32_t sc = 0;
+    uint32_t sc = 0, ic = 0;
     if (lane == 0) {
-      for (int item = blockIdx.x; item < pl.items && ok; item += gridDim.x) {
+      for (int item = blockIdx.x; item < pl.items && ok; item += gridDim.x, ++ic) {
         const int bh = item / pl.row_blocks;
-        for (int pass = 0; pass < pl.passes && ok; ++pass)
-          for (int g = 0; g < pl.groups && ok; ++g)
-            for (int c = 0; c < kChunks && ok; ++c)
-              for (int t = 0; t < kGroupTiles && ok; ++t) {
-                const int s = sc % kStages;
-                if (!(ok = mbar_wait(&ms->stage_empty[s], ((sc / kStages) & 1) ^ 1, wc))) break;
-                mbar_arrive_expect_tx(&ms->raw_full[s], kHalfBytes);
-                tma_load_3d(smem + s * kStageBytes, &tm_k, &ms->raw_full[s], c * kChunkD, g * kGroupKeys + t * kTileN,
-                            bh);
-                ++sc;
-              }
+        bool slow = false;
+        int total = pl.total(false);
+        for (int p = 0; p < total && ok; ++p) {
+          if (pl.general && p == 3) {
+            if (!(ok = mbar_wait(&ms->plan, ic & 1, wc))) break;
+            slow = *plan_slow != 0;
+            total = pl.total(slow);
+          }
+          const int kind = pl.kind(p, slow), nt = pl.ntiles(kind);
+          for (int pos = 0; pos < nt && ok; ++pos) {
+            const int tile = tile_of(pos, nt);
+            for (int c = 0; c < kChunks && ok; ++c) {
+              const int s = sc % kStages;
+              if (!(ok = mbar_wait(&ms->stage_empty[s], ((sc / kStages) & 1) ^ 1, wc))) break;
+              mbar_arrive_expect_tx(&ms->raw_full[s], kHalfBytes);
+              if (kind == kSample)
+                tma_load_3d(smem + s * kStageBytes, &tm_s, &ms->raw_full[s], c * kChunkD, 0, bh);
+              else
+                tma_load_3d(smem + s * kStageBytes, &tm_k, &ms->raw_full[s], c * kChunkD, tile * kTileN, bh);
+              ++sc;
+            }
+          }
+        }
       }
       if (!ok) {
         *abort_flag = 1;
@@ -191,45 +429,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------- MMA
     bool ok = true;
     if (lane == 0) {
-      uint32_t sc = 0, gc = 0, ic = 0;
+      uint32_t sc = 0, ic = 0, dc0 = 0, dc1 = 0;  // accumulators used so far
       for (int item = blockIdx.x; item < pl.items && ok; item += gridDim.x, ++ic) {
         if (!(ok = mbar_wait(&ms->q_ready, ic & 1, wc))) break;
-        for (int pass = 0; pass < pl.passes && ok; ++pass)
-          for (int g = 0; g < pl.groups && ok; ++g, ++gc) {
-            if (!(ok = mbar_wait(&ms->d_empty, (gc & 1) ^ 1, wc))) break;
+        bool slow = false;
+        int total = pl.total(false);
+        for (int p = 0; p < total && ok; ++p) {
+          if (pl.general && p == 3) {
+            if (!(ok = mbar_wait(&ms->plan, ic & 1, wc))) break;
+            slow = *plan_slow != 0;
+            total = pl.total(slow);
+          }
+          const int kind = pl.kind(p, slow), nt = pl.ntiles(kind);
+          const bool three = kind != kSample;  // the sample needs hi.hi only
+          for (int pos = 0; pos < nt && ok; ++pos) {
+            const int b = pos & 1;
+            if (!(ok = mbar_wait(&ms->d_empty[b], ((b ? dc1 : dc0) & 1) ^ 1, wc))) break;
             tc_fence_after();
-            for (int c = 0; c < kChunks && ok; ++c, sc += kGroupTiles) {
-              // the chunk's two stages (tile 0, tile 1) are consecutive in the ring
-              const int s0 = sc % kStages, s1 = (sc + 1) % kStages;
-              if (!(ok = mbar_wait(&ms->conv_full[s0], (sc / kStages) & 1, wc) &&
-                         mbar_wait(&ms->conv_full[s1], ((sc + 1) / kStages) & 1, wc)))
-                break;
+            const uint32_t d = tmem + kColD + (uint32_t)b * kTileN;
+            for (int c = 0; c < kChunks && ok; ++c, ++sc) {
+              const int s = sc % kStages;
+              if (!(ok = mbar_wait(&ms->conv_full[s], (sc / kStages) & 1, wc))) break;
               tc_fence_after();
-              const uint32_t st_addr[2] = {smem_addr(smem + s0 * kStageBytes), smem_addr(smem + s1 * kStageBytes)};
+              const uint32_t st = smem_addr(smem + s * kStageBytes);
+              const uint64_t bhi0 = smem_desc(st, 16, 1024, kSwizzle128B);
+              const uint64_t blo0 = smem_desc(st + kHalfBytes, 16, 1024, kSwizzle128B);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
                 const uint32_t ks = (uint32_t)(c * 4 + kk);  // K-step of 8 channels
                 const uint32_t ahi = tmem + kColQhi + ks * 8, alo = tmem + kColQlo + ks * 8;
-                const uint32_t first = (c == 0 && kk == 0) ? 0u : 1u;
                 // +32 bytes per K-step inside the 128-byte row = +2 in the address field
-                uint64_t bhi[2], blo[2];
-#pragma unroll
-                for (int t = 0; t < kGroupTiles; ++t) {
-                  bhi[t] = smem_desc(st_addr[t], 16, 1024, kSwizzle128B) + (uint64_t)(kk * 2);
-                  blo[t] = smem_desc(st_addr[t] + kHalfBytes, 16, 1024, kSwizzle128B) + (uint64_t)(kk * 2);
+                const uint64_t bhi = bhi0 + (uint64_t)(kk * 2), blo = blo0 + (uint64_t)(kk * 2);
+                umma_tf32_ts(d, ahi, bhi, (c == 0 && kk == 0) ? 0u : 1u);
+                if (three) {
+                  umma_tf32_ts(d, ahi, blo, 1u);
+                  umma_tf32_ts(d, alo, bhi, 1u);
                 }
-#pragma unroll
-                for (int t = 0; t < kGroupTiles; ++t) umma_tf32_ts(tmem + kColD + t * kTileN, ahi, bhi[t], first);
-#pragma unroll
-                for (int t = 0; t < kGroupTiles; ++t) umma_tf32_ts(tmem + kColD + t * kTileN, ahi, blo[t], 1u);
-#pragma unroll
-                for (int t = 0; t < kGroupTiles; ++t) umma_tf32_ts(tmem + kColD + t * kTileN, alo, bhi[t], 1u);
               }
-              umma_commit(&ms->stage_empty[s0]);
-              umma_commit(&ms->stage_empty[s1]);
+              umma_commit(&ms->stage_empty[s]);
             }
-            if (ok) umma_commit(&ms->d_full);
+            if (ok) {
+              umma_commit(&ms->d_full[b]);
+              (b ? dc1 : dc0) += 1;
+            }
           }
+        }
         if (ok) umma_commit(&ms->q_empty);
       }
     }
@@ -245,53 +489,78 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------- converters
     const int tid = threadIdx.x - 128;
-    uint32_t sc = 0;
+    uint32_t sc = 0, ic = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < pl.items && ok; item += gridDim.x)
-      for (int pass = 0; pass < pl.passes && ok; ++pass)
-        for (int g = 0; g < pl.groups && ok; ++g)
-          for (int c = 0; c < kChunks * kGroupTiles && ok; ++c, ++sc) {
-            const int s = sc % kStages;
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ms->raw_full[s], (sc / kStages) & 1, wc)))) break;
-            uint4* hi = reinterpret_cast<uint4*>(smem + s * kStageBytes);
-            uint4* lo = reinterpret_cast<uint4*>(smem + s * kStageBytes + kHalfBytes);
+    for (int item = blockIdx.x; item < pl.items && ok; item += gridDim.x, ++ic) {
+      bool slow = false;
+      int total = pl.total(false);
+      for (int p = 0; p < total && ok; ++p) {
+        if (pl.general && p == 3) {
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ms->plan, ic & 1, wc)))) break;
+          slow = *plan_slow != 0;
+          total = pl.total(slow);
+        }
+        const int n_stages = pl.ntiles(pl.kind(p, slow)) * kChunks;
+        for (int q = 0; q < n_stages && ok; ++q, ++sc) {
+          const int s = sc % kStages;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ms->raw_full[s], (sc / kStages) & 1, wc)))) break;
+          uint4* hi = reinterpret_cast<uint4*>(smem + s * kStageBytes);
+          uint4* lo = reinterpret_cast<uint4*>(smem + s * kStageBytes + kHalfBytes);
 #pragma unroll 4
-            for (int e = tid; e < kHalfBytes / 16; e += 128) {
-              const uint4 v = hi[e];
-              const uint4 h = make_uint4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
-              hi[e] = h;
-              lo[e] = make_uint4(__float_as_uint(__uint_as_float(v.x) - __uint_as_float(h.x)),
-                                 __float_as_uint(__uint_as_float(v.y) - __uint_as_float(h.y)),
-                                 __float_as_uint(__uint_as_float(v.z) - __uint_as_float(h.z)),
-                                 __float_as_uint(__uint_as_float(v.w) - __uint_as_float(h.w)));
-            }
-            fence_proxy_async_smem();  // the pieces are read by the tensor core
-            mbar_arrive(&ms->conv_full[s]);
+          for (int e = tid; e < kHalfBytes / 16; e += 128) {
+            const uint4 v = hi[e];
+            const uint4 h = make_uint4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
+            hi[e] = h;
+            lo[e] = make_uint4(__float_as_uint(__uint_as_float(v.x) - __uint_as_float(h.x)),
+                               __float_as_uint(__uint_as_float(v.y) - __uint_as_float(h.y)),
+                               __float_as_uint(__uint_as_float(v.z) - __uint_as_float(h.z)),
+                               __float_as_uint(__uint_as_float(v.w) - __uint_as_float(h.w)));
           }
+          fence_proxy_async_smem();  // the pieces are read by the tensor core
+          mbar_arrive(&ms->conv_full[s]);
+        }
+      }
+    }
     if (!ok && threadIdx.x == 128) *abort_flag = 1;
   } else if (warp >= 8) {
     // ------------------------------------------------------------- selectors
+    const int wg = (warp - 8) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // TMEM lane = query block of the item
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-    uint16_t* hist = reinterpret_cast<uint16_t*>(smem + kOffHist);  // [bin][row]
-    uint32_t gc = 0, ic = 0;
+    uint16_t* hist_row = reinterpret_cast<uint16_t*>(smem + kOffHist) + r;  // + bin * kRows
+    Row R;
+    R.nblk = a.nblk;
+    R.hw = reinterpret_cast<uint32_t*>(smem + kOffHist) + (r >> 1);
+    R.inc = 1u << ((r & 1) * 16);
+    R.cand_s = reinterpret_cast<float*>(smem + kOffHist) + wg * kCap * kRows + r;
+    R.cand_j = reinterpret_cast<uint16_t*>(smem + kOffCandJ) + wg * kCap * kRows + r;
+    R.desc = wg == 1;
+    R.cap = a.K_capacity;
+    R.stride = pl.stride;
+    R.ns = pl.ns;
+    // normal quantile of the kept fraction of the off-diagonal blocks
+    const float zq = pl.general ? normcdfinvf(1.0f - (float)(a.keep - 1) / (float)(a.nblk - 1)) : 0.0f;
+    uint32_t tc = 0, ic = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < pl.items && ok; item += gridDim.x, ++ic) {
+    for (int item = blockIdx.x; item < pl.items; item += gridDim.x, ++ic) {
       const int bh = item / pl.row_blocks;
-      const int i = (item - bh * pl.row_blocks) * kRows + r;  // my query block
-      const bool row = i < a.nblk;
-      // ---- my query block's mean, split into tf32 pieces, into my TMEM lane
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ms->q_empty, (ic & 1) ^ 1, wc)))) break;
-      tc_fence_after();
-      {
-        const float4* qrow = reinterpret_cast<const float4*>(a.q_bar + ((size_t)bh * a.nblk + (row ? i : 0)) * kHeadDim);
+      const int rb = item - bh * pl.row_blocks;
+      R.i = rb * kRows + r;
+      R.row = R.i < a.nblk;
+      // ---- my query block's mean (my warpgroup's 64 channels), split into
+      // tf32 pieces, into my TMEM lane
+      ok = ok && __all_sync(0xffffffffu, mbar_wait(&ms->q_empty, (ic & 1) ^ 1, wc));
+      if (ok) {
+        tc_fence_after();
+        const float4* qrow = reinterpret_cast<const float4*>(a.q_bar + ((size_t)bh * a.nblk + (R.row ? R.i : 0)) * kHeadDim) +
+                             wg * 16;
 #pragma unroll 1
-        for (int part = 0; part < 4; ++part) {
+        for (int part = 0; part < 2; ++part) {
           uint32_t hv[32], lv[32];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float4 v = row ? __ldg(qrow + part * 8 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 v = R.row ? __ldg(qrow + part * 8 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
             const float f[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -300,114 +569,199 @@ __global__ void __launch_bounds__(kThreads, 1)
               lv[4 * e + k] = __float_as_uint(f[k] - __uint_as_float(h));
             }
           }
-          tmem_st_32cols(lane_addr + kColQhi + part * 32, hv);
-          tmem_st_32cols(lane_addr + kColQlo + part * 32, lv);
+          const uint32_t col = (uint32_t)(wg * 64 + part * 32);
+          tmem_st_32cols(lane_addr + kColQhi + col, hv);
+          tmem_st_32cols(lane_addr + kColQlo + col, lv);
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&ms->q_ready);
       }
+      if (!(ok = sel_and(ok))) break;
       // ---- selection state of my row
-      uint32_t prefix = 0, mask = 0;
-      int remaining = a.keep - 1;  // off-diagonal blocks to keep (budget mode)
-      int shift = 24;
-      int32_t* out = a.kept_idx + ((size_t)bh * a.nblk + (row ? i : 0)) * a.K_capacity;
-      float* srow = a.scores != nullptr && row ? a.scores + ((size_t)bh * a.nblk + i) * a.nblk : nullptr;
-      int written = 0, eq_taken = 0;
-      bool output = false;
-      // per element of a chunk of my score row: count its digit (radix pass,
-      // fire-and-forget shared-memory atomic on my 16-bit half of a word; the
-      // neighbouring row owns the other half) or decide and write it (output)
-      const uint32_t inc = 1u << ((r & 1) * 16);
-      uint32_t* hw = reinterpret_cast<uint32_t*>(smem + kOffHist) + (r >> 1);  // + bin * 64
-      auto scan_chunk = [&](const uint32_t (&v)[32], int j0) {
-        if (!output) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int j = j0 + e;
-            const uint32_t key = order_key(__uint_as_float(v[e]));
-            if (j < a.nblk && j != i && (key & mask) == prefix) atomicAdd(hw + ((key >> shift) & 0xFFu) * 64, inc);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int j = j0 + e;
-            if (j >= a.nblk) continue;  // (fully unrolled: v stays in registers)
-            const float sv = __uint_as_float(v[e]);
-            const uint32_t key = order_key(sv);
-            if (srow != nullptr) srow[j] = sv;
-            bool take;
-            if (j == i) {
-              take = true;
-            } else if (a.threshold_mode) {
-              take = sv >= a.tau;
-            } else if (a.keep <= 1) {
-              take = false;
-            } else if (a.keep >= a.nblk) {
-              take = true;
-            } else {
-              take = key > prefix || (key == prefix && eq_taken < remaining);
-              if (key == prefix && take) ++eq_taken;
-            }
-            if (take && written < a.K_capacity) out[written++] = j;  // bounded by the row's capacity
-          }
+      int need = a.keep - 1;  // off-diagonal blocks still to place (budget form)
+      if (a.threshold_mode) {
+        R.cs = a.tau;
+        R.cj = 0xFFFF;
+      } else if (a.keep <= 1) {
+        R.cs = __int_as_float(0x7f800000);  // +inf: nothing but the diagonal
+        R.cj = -1;
+      } else {
+        R.cs = __int_as_float(0xff800000);  // -inf: everything (general rows set their cut later)
+        R.cj = 0xFFFF;
+      }
+      R.A = 0.0f;
+      R.B = 0.0f;
+      R.tb = 0;
+      R.kpre = R.kmask = R.vpre = R.vmask = 0;
+      R.sh = 24;
+      R.vlevel = false;
+      R.n = 0;
+      R.w = 0;
+      R.top = a.threshold_mode ? a.K_capacity - 1 : a.keep - 1;
+      R.out = a.kept_idx + ((size_t)bh * a.nblk + (R.row ? R.i : 0)) * a.K_capacity;
+      R.srow = a.scores != nullptr && R.row ? a.scores + ((size_t)bh * a.nblk + R.i) * a.nblk : nullptr;
+      R.sum = R.sq = 0.0f;
+      R.ns_seen = 0;
+      bool slow = false;
+      int total = pl.total(false);
+      for (int p = 0; p < total; ++p) {
+        const int kind = pl.kind(p, slow), nt = pl.ntiles(kind);
+        const int mine = wg == 0 ? (nt + 1) / 2 : nt / 2;
+        if (kind == kLevel) {
+          const int lvl = p - 2;
+          R.vlevel = lvl >= 4;
+          R.sh = R.vlevel ? (uint32_t)(8 - 8 * (lvl - 4)) : (uint32_t)(24 - 8 * lvl);
         }
-      };
-      for (int pass = 0; pass < pl.passes && ok; ++pass) {
-        output = pass == pl.passes - 1;
-        for (int g = 0; g < pl.groups && ok; ++g, ++gc) {
-          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ms->d_full, gc & 1, wc)))) break;
+        for (int k = 0; k < mine && ok; ++k) {
+          const int tile = wg == 0 ? k : nt - 1 - k;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ms->d_full[wg], tc & 1, wc)))) break;
           tc_fence_after();
-          // the group's 256 scores in eight 32-column chunks; the load of the
-          // next chunk is in flight while one is processed
-          uint32_t va[32], vb[32];
-          tmem_ld_32cols(lane_addr + kColD, va);
-#pragma unroll 1
-          for (int part = 0; part < kGroupKeys / 32; part += 2) {
-            tmem_wait_ld_regs(va);
-            tmem_ld_32cols(lane_addr + kColD + (part + 1) * 32, vb);
-            if (row) scan_chunk(va, g * kGroupKeys + part * 32);
-            tmem_wait_ld_regs(vb);
-            if (part + 2 < kGroupKeys / 32) tmem_ld_32cols(lane_addr + kColD + (part + 2) * 32, va);
-            if (row) scan_chunk(vb, g * kGroupKeys + (part + 1) * 32);
+          const uint32_t d = lane_addr + kColD + (uint32_t)wg * kTileN;
+          const int jbase = tile * kTileN;
+          const bool checks = kind == kSample || tile == rb || jbase + kTileN > a.nblk;
+          switch (kind) {
+            case kSample: scan_tile<kSample>(d, 0, true, R); break;
+            case kHist: scan_tile<kHist>(d, jbase, checks, R); break;
+            case kCompact: scan_tile<kCompact>(d, jbase, checks, R); break;
+            case kLevel: scan_tile<kLevel>(d, jbase, checks, R); break;
+            default: scan_tile<kOutput>(d, jbase, checks, R); break;
           }
           tc_fence_before();
-          mbar_arrive(&ms->d_empty);
+          mbar_arrive(&ms->d_empty[wg]);
+          ++tc;
         }
-        if (!ok) break;
-        if (!output && row) {
-          // ---- the digit of the remaining-th largest among the matching keys;
-          // clear the bins for the next pass
-          int cum = 0, digit = -1, above = 0;
-#pragma unroll 4
-          for (int b = kBins - 1; b >= 0; --b) {
-            uint16_t* h = hist + b * kRows + r;
-            const int cnt = *h;
-            *h = 0;
-            if (digit < 0) {
-              if (cum + cnt >= remaining) {
-                digit = b;
-                above = cum;
-              } else {
-                cum += cnt;
-              }
+        if (!(ok = sel_and(ok))) break;  // also: every atomic and slot of the pass is done
+        // ---- end of pass
+        if (kind == kSample) {
+          if (wg == 0) {
+            if (R.row) {
+              const float cnt = (float)(R.ns_seen > 0 ? R.ns_seen : 1);
+              const float mean = R.sum / cnt;
+              const float sd = sqrtf(fmaxf(R.sq / cnt - mean * mean, 0.0f));
+              const float lo = mean + (zq - kWindowSd) * sd;
+              float A = 127.0f / (kWindowSd * sd);  // 254 bins across 2 * kWindowSd * sd
+              float B = 1.0f - lo * A;
+              if (!(sd > 0.0f) || !isfinite(A) || !isfinite(B)) A = B = 0.0f;  // one bin: the fallback decides
+              ms->bin_a[r] = A;
+              ms->bin_b[r] = B;
             }
           }
-          prefix |= (uint32_t)digit << shift;
-          mask |= 0xFFu << shift;
-          remaining -= above;
-          shift -= 8;
+          sel_sync();
+          R.A = ms->bin_a[r];
+          R.B = ms->bin_b[r];
+        } else if (kind == kHist) {
+          bool bad = false;
+          if (wg == 0 && R.row) {
+            int above, cnt;
+            const int b = find_bin(hist_row, need, above, cnt);
+            R.tb = b < 0 ? 0u : (uint32_t)b;
+            need -= above;
+            bad = b < 0 || cnt > kCap;
+            ms->tb[r] = (int)R.tb;
+          }
+          slow = sel_or(bad);
+          if (wg == 0 && r == 0) {
+            *plan_slow = slow ? 1 : 0;
+            mbar_arrive(&ms->plan);
+          }
+          total = pl.total(slow);
+          R.tb = (uint32_t)ms->tb[r];
+        } else if (kind == kCompact) {
+          if (wg == 1) ms->n1[r] = R.n;
+          sel_sync();
+          if (wg == 0 && R.row) {
+            float* s0 = R.cand_s;                    // my slots, then the second warpgroup's
+            uint16_t* j0 = R.cand_j;
+            float* s1 = R.cand_s + kCap * kRows;
+            uint16_t* j1 = R.cand_j + kCap * kRows;
+            const int n0 = min(R.n, kCap), n1 = min(ms->n1[r], kCap), tot = n0 + n1;
+            R.cs = __int_as_float(0x7f800000);
+            R.cj = -1;
+            for (int x = 0; x < tot; ++x) {
+              const float sx = x < n0 ? s0[x * kRows] : s1[(x - n0) * kRows];
+              const int jx = x < n0 ? j0[x * kRows] : j1[(x - n0) * kRows];
+              int rank = 0;  // candidates before x in (score desc, index asc) order
+              for (int y = 0; y < tot; ++y) {
+                const float sy = y < n0 ? s0[y * kRows] : s1[(y - n0) * kRows];
+                const int jy = y < n0 ? j0[y * kRows] : j1[(y - n0) * kRows];
+                rank += (sy > sx || (sy == sx && jy < jx)) ? 1 : 0;
+              }
+              if (rank == need - 1) {
+                R.cs = sx;
+                R.cj = jx;
+                break;
+              }
+            }
+            for (int x = 0; x < n0; ++x) {
+              s0[x * kRows] = 0.0f;
+              j0[x * kRows] = 0;
+            }
+            for (int x = 0; x < n1; ++x) {
+              s1[x * kRows] = 0.0f;
+              j1[x * kRows] = 0;
+            }
+            ms->cut_s[r] = R.cs;
+            ms->cut_j[r] = R.cj;
+          }
+          sel_sync();
+          R.cs = ms->cut_s[r];
+          R.cj = ms->cut_j[r];
+        } else if (kind == kLevel) {
+          if (wg == 0 && R.row) {
+            int above, cnt;
+            int b = find_bin(hist_row, need, above, cnt);
+            if (b < 0) b = 0;
+            need -= above;
+            if (R.vlevel) {
+              R.vpre |= (uint32_t)b << R.sh;
+              R.vmask |= 0xFFu << R.sh;
+            } else {
+              R.kpre |= (uint32_t)b << R.sh;
+              R.kmask |= 0xFFu << R.sh;
+            }
+            ms->kpre[r] = R.kpre;
+            ms->kmask[r] = R.kmask;
+            ms->vpre[r] = R.vpre;
+            ms->vmask[r] = R.vmask;
+            if (p == 1 + kLevels) {  // the last level: key and index of the cut are fixed
+              ms->cut_s[r] = key_value(R.kpre);
+              ms->cut_j[r] = (int)(0xFFFFu - R.vpre);
+            }
+          }
+          sel_sync();
+          R.kpre = ms->kpre[r];
+          R.kmask = ms->kmask[r];
+          R.vpre = ms->vpre[r];
+          R.vmask = ms->vmask[r];
+          if (p == 1 + kLevels) {
+            R.cs = ms->cut_s[r];
+            R.cj = ms->cut_j[r];
+          }
+        } else {  // kOutput
+          (wg == 0 ? ms->w0 : ms->w1)[r] = R.w;
+          sel_sync();
+          if (R.row) {
+            const int w0 = ms->w0[r], w1 = ms->w1[r];
+            const int written = min(w0 + w1, a.K_capacity);
+            if (wg == 0) {
+              a.kept_cnt[(size_t)bh * a.nblk + R.i] = written;
+            } else {
+              if (a.threshold_mode && w1 > 0 && w0 + w1 <= a.K_capacity) {
+                // my blocks sit at the end of the row: move them behind the first warpgroup's
+                const int src = a.K_capacity - w1;
+                for (int e = 0; e < w1 && src != w0; ++e) R.out[w0 + e] = R.out[src + e];
+              }
+              for (int e = a.threshold_mode ? written : a.keep; e < a.K_capacity; ++e) R.out[e] = -1;
+            }
+          }
         }
       }
       if (!ok) break;
-      if (row) {
-        for (int e = written; e < a.K_capacity; ++e) out[e] = -1;
-        a.kept_cnt[(size_t)bh * a.nblk + i] = written;
-      }
     }
     if (!ok) {
       tmem_wait_ld();
-      if (r == 0) *abort_flag = 1;
+      *abort_flag = 1;
     }
   }
 
@@ -423,17 +777,18 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-// [B*H, nblk, 128] fp32 seen as 3-D (d, key block, batch-head); a box is 32
-// channels x 128 key blocks, 128-byte swizzle; key blocks past nblk read 0.
-int make_pooled_map(CUtensorMap* map, const float* base, int nblk, int BH) {
+// [B*H, nblk, 128] fp32 seen as 3-D (d, key block, batch-head), every
+// `stride`-th key block from block 0 (rows = ceil(nblk / stride)); a box is
+// 32 channels x 128 rows, 128-byte swizzle; rows past the end read 0.
+int make_pooled_map(CUtensorMap* map, const float* base, int nblk, int BH, int stride) {
   void* p = nullptr;
   cudaDriverEntryPointQueryResult qr;
   if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) != cudaSuccess ||
       qr != cudaDriverEntryPointSuccess || p == nullptr)
     return SBATTN_ERR_CUDA;
   EncodeTiledFn fn = reinterpret_cast<EncodeTiledFn>(p);
-  const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)nblk, (cuuint64_t)BH};
-  const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 4, (cuuint64_t)nblk * kHeadDim * 4};
+  const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)((nblk + stride - 1) / stride), (cuuint64_t)BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)stride * kHeadDim * 4, (cuuint64_t)nblk * kHeadDim * 4};
   const cuuint32_t box[3] = {(cuuint32_t)kChunkD, (cuuint32_t)kTileN, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, estr,
@@ -449,9 +804,12 @@ int select_max_nblk() { return 65535; }  // u16 histogram counts
 int launch_select(const SelectArgs& a, cudaStream_t stream) {
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   if (a.nblk > select_max_nblk()) return SBATTN_ERR_UNSUPPORTED_SHAPE;
-  CUtensorMap map;
-  int rc = make_pooled_map(&map, a.k_bar, a.nblk, a.B * a.H);
+  CUtensorMap map, sample_map;
+  int rc = make_pooled_map(&map, a.k_bar, a.nblk, a.B * a.H, 1);
   if (rc != SBATTN_OK) return rc;
+  // the sample pass: every ceil(nblk/128)-th key block, at most 128 of them
+  if ((rc = make_pooled_map(&sample_map, a.k_bar, a.nblk, a.B * a.H, (a.nblk + kTileN - 1) / kTileN)) != SBATTN_OK)
+    return rc;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -459,7 +817,7 @@ int launch_select(const SelectArgs& a, cudaStream_t stream) {
     return SBATTN_ERR_CUDA;
   const long items = (long)a.B * a.H * ((a.nblk + kRows - 1) / kRows);
   const int grid = (int)(items < sms ? items : sms);
-  select_kernel<<<grid, kThreads, kSmemBytes, stream>>>(map, a, kWaitLimitNs);
+  select_kernel<<<grid, kThreads, kSmemBytes, stream>>>(map, sample_map, a, kWaitLimitNs);
   return cudaGetLastError() == cudaSuccess ? SBATTN_OK : SBATTN_ERR_CUDA;
 }
 
