@@ -26,23 +26,29 @@
 //     wrote it) and lo (a second buffer with the same swizzled positions).
 //   * The tiles of a pass alternate between the two selector warpgroups: the
 //     first takes tiles 0, 1, 2, ... (accumulator 0), the second tiles T-1,
-//     T-2, ... (accumulator 1), so that each writes its kept blocks in order
-//     from its own end of the output row.
+//     T-2, ... (accumulator 1).
 // Exact top-K per row, in four passes over the scores:
 //   1. sample: one tile of every ceil(nblk/128)-th key block, one product
 //      (hi.hi); mean m and deviation sd of the row's sampled scores place a
-//      window of 2 sd around m + z sd, z the normal quantile of the kept
+//      window of 1.5 sd around m + z sd, z the normal quantile of the kept
 //      fraction;
-//   2. histogram: 256 bins, 254 across the window and one for each side,
-//      bin(s) = round(clamp(s * A + B, 0, 255)), a non-decreasing function of
-//      s; the bin holding the (K-1)-th largest off-diagonal score follows from
-//      the counts (u16 per row in shared memory, fire-and-forget atomics);
+//   2. histogram: 128 bins, bin(s) = round(clamp(s * A + B, 0, 127)), a
+//      non-decreasing function of s; bins 1 .. 126 cover the window, 0 and
+//      127 everything below and above it; u32 counts per row in shared
+//      memory (a warp's 32 rows hit 32 banks) by adds without a result and
+//      without a branch; the bin holding the (K-1)-th largest off-diagonal
+//      score follows from the counts;
 //   3. compaction: the scores of that bin (a few dozen at most) go to
 //      shared memory with their block index; the (K-1)-th largest under the
 //      order (score descending, block index ascending) among them is the cut;
-//   4. output: the diagonal and every block at or above the cut, in
-//      ascending block order.
-// If some row's bin holds more than 32 blocks (a sample that misplaced the
+//   4. output: the diagonal and every block at or above the cut.  For nblk
+//      <= 4096 each thread sets one bit per kept block in a shared-memory
+//      bitmask; at the next item's start (while the tensor core begins that
+//      item) the selector warps write the rows, word by word, a word's kept
+//      blocks in one store of consecutive entries.  Beyond 4096 each
+//      warpgroup writes its own tiles' blocks from its end of the row (the
+//      first forward, the second backward from the last position).
+// If some row's bin holds more than 40 blocks (a sample that misplaced the
 // window, or mass ties), the item runs instead six radix levels restricted to
 // that bin: the four bytes of an order-preserving key of the score, then the
 // two bytes of (65535 - block index), which fixes the cut exactly.  Threshold
@@ -52,6 +58,8 @@
 //   warp 0: TMA producer           warp 1: TMEM allocator + MMA issuer
 //   warps 4-7: converters          warps 8-15: two selector warpgroups
 //                                  (TMEM lane quarter = warp % 4)
+// The producer warpgroups give up registers (72 per thread) to the selector
+// warpgroups (184), whose chunk code is unrolled over 32 scores.
 // Every mbarrier wait is bounded; a failed wait is shared with the other
 // selector warpgroup at the next named barrier, after which the kernel stores
 // nothing more, lets its own copies and MMAs finish, frees TMEM and returns.
@@ -69,19 +77,32 @@ constexpr int kChunks = kHeadDim / kChunkD;   // 4
 constexpr int kStages = 4;                    // a stage: one tile x one chunk of 32 channels
 constexpr int kHalfBytes = kTileN * kChunkD * 4;      // 16 KB: hi (TMA target) or lo
 constexpr int kStageBytes = 2 * kHalfBytes;
+// One 64 KB region of shared memory, zero between uses, serves in turn as
+//   * the window histogram: u32 counts [bin][row], 128 bins (a warp's 32
+//     rows hit 32 banks whatever their bins);
+//   * the candidates of the boundary bin: f32 scores [wg][slot][row], then
+//     u16 block indices [wg][slot][row];
+//   * the kept-block bitmask: u32 words [word][row ^ (word % 32)], 32 blocks
+//     per word (nblk <= 4096); the xor spreads both a warp's 32 rows of one
+//     word and one row's 32 words over the 32 banks;
+//   * the fallback's byte histograms: u16 counts [digit][row], 256 digits.
+constexpr int kWinBins = 128;
 constexpr int kBins = 256;
-constexpr int kHistBytes = kBins * kRows * 2;         // u16 counts, [bin][row]
+constexpr int kHistBytes = kBins * kRows * 2;         // 64 KB
 constexpr int kOffHist = kStages * kStageBytes;       // 128 KB
-constexpr int kCap = 32;                              // candidates per row and selector warpgroup
-// candidates reuse the (then zero) histogram space: f32 scores [wg][slot][row],
-// then u16 block indices [wg][slot][row]
+constexpr int kCap = 40;                              // candidates per row and selector warpgroup
 constexpr int kOffCandJ = kOffHist + 2 * kCap * kRows * 4;
-static_assert(kOffCandJ + 2 * kCap * kRows * 2 <= kOffHist + kHistBytes, "candidates fit the histogram space");
+static_assert(kOffCandJ + 2 * kCap * kRows * 2 <= kOffHist + kHistBytes, "candidates fit the shared region");
+static_assert(kWinBins * kRows * 4 <= kHistBytes, "window histogram fits the shared region");
+constexpr int kMaskWords = kHistBytes / (kRows * 4);  // 128 words: 4096 blocks per row
 constexpr int kOffMisc = kOffHist + kHistBytes;       // 192 KB
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColQhi = 0, kColQlo = 128, kColD = 256;  // accumulator b at kColD + 128 b
 constexpr int kLevels = 6;                    // fallback: 4 key bytes + 2 index bytes
-constexpr float kWindowSd = 1.0f;             // half-width of the histogram window, in sd
+constexpr float kWindowSd = 0.75f;            // half-width of the histogram window, in sd
+// registers: the selectors' unrolled chunk code takes the producers' share
+constexpr uint32_t kRegsProducers = 72, kRegsSelectors = 184;
+static_assert(256 * kRegsProducers + 256 * kRegsSelectors == kThreads * 128, "register split = 512 x 128");
 
 enum PassKind { kSample = 0, kHist = 1, kCompact = 2, kLevel = 3, kOutput = 4 };
 
@@ -98,7 +119,7 @@ struct Misc {
   float bin_a[kRows], bin_b[kRows], cut_s[kRows];
   int cut_j[kRows], tb[kRows];
   uint32_t kpre[kRows], kmask[kRows], vpre[kRows], vmask[kRows];
-  int n1[kRows], w0[kRows], w1[kRows];
+  int n0[kRows], n1[kRows], need[kRows], w0[kRows], w1[kRows];
 };
 constexpr int kSmemBytes = kOffMisc + (int)sizeof(Misc);
 
@@ -156,15 +177,18 @@ SB_DEV uint32_t order_key(float f) {
 }
 SB_DEV float key_value(uint32_t k) { return __uint_as_float((k & 0x80000000u) ? (k ^ 0x80000000u) : ~k); }
 
-// Histogram bin of a score: round(clamp(s * A + B, 0, 255)).  Each step is
-// non-decreasing in s (fma, min, max, and rounding to an integer by adding
-// 1.5 * 2^23), so a higher bin means a strictly higher score.
+// Window bin of a score: round(clamp(s * A + B, 0, 127)).  The window maps
+// to bins 1 .. 126; bin 0 holds everything below it and bin 127 everything
+// above.  Each step is non-decreasing in s (fma, max, min, and rounding to an
+// integer by adding 1.5 * 2^23), so a higher bin means a strictly higher
+// score.
 SB_DEV uint32_t bin_of(float s, float A, float B) {
-  const float x = fminf(fmaxf(fmaf(s, A, B), 0.0f), 255.0f);
-  return __float_as_uint(x + 12582912.0f) & 0xFFu;
+  const float x = fminf(fmaxf(fmaf(s, A, B), 0.0f), 127.0f);
+  return __float_as_uint(x + 12582912.0f) & 0x7Fu;
 }
 
 SB_DEV uint32_t tf32_hi(uint32_t u) { return u & 0xFFFFE000u; }
+
 
 // The schedule every role walks: work items (128 query blocks of one
 // batch-head) strided over the grid, passes, the tiles of a pass (in the
@@ -172,6 +196,7 @@ SB_DEV uint32_t tf32_hi(uint32_t u) { return u & 0xFFFFE000u; }
 struct Plan {
   int items, row_blocks, tiles, stride, ns;
   bool general;  // budget form with 1 < keep < nblk
+  bool bitmask;  // kept blocks gathered in shared memory, written row by row
   SB_DEV void init(const SelectArgs& a) {
     row_blocks = (a.nblk + kRows - 1) / kRows;
     items = a.B * a.H * row_blocks;
@@ -179,6 +204,7 @@ struct Plan {
     stride = (a.nblk + kTileN - 1) / kTileN;  // sampled blocks: j = m * stride, m < ns <= 128
     ns = (a.nblk + stride - 1) / stride;
     general = !a.threshold_mode && a.keep > 1 && a.keep < a.nblk;
+    bitmask = a.nblk <= kMaskWords * 32;
   }
   SB_DEV int total(bool slow) const { return general ? (slow ? 3 + kLevels : 4) : 1; }
   SB_DEV int kind(int p, bool slow) const {
@@ -194,20 +220,48 @@ struct Plan {
 // descend from the last tile.
 SB_DEV int tile_of(int pos, int tiles) { return (pos & 1) ? tiles - 1 - (pos >> 1) : (pos >> 1); }
 
+// Shared-memory stores and adds on 32-bit shared addresses (no address-space
+// conversion per element); the add returns nothing, so nothing waits for it.
+SB_DEV void sts_u32(uint32_t a, uint32_t v) { asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory"); }
+SB_DEV void sts_u16(uint32_t a, uint32_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"((unsigned short)v) : "memory");
+}
+SB_DEV void red_add(uint32_t a, uint32_t v) { asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory"); }
+// Stores under a predicate, with no branch around them (a divergent branch
+// per element costs more than the work it skips).
+SB_DEV void stg_s32_if(bool p, int32_t* a, int32_t v) {
+  asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %2, 0;\n\t@q st.global.s32 [%0], %1;\n\t}\n" ::"l"(a), "r"(v),
+               "r"((uint32_t)p)
+               : "memory");
+}
+SB_DEV void sts_u32_if(bool p, uint32_t a, uint32_t v) {
+  asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %2, 0;\n\t@q st.shared.u32 [%0], %1;\n\t}\n" ::"r"(a), "r"(v),
+               "r"((uint32_t)p)
+               : "memory");
+}
+SB_DEV void sts_u16_if(bool p, uint32_t a, uint32_t v) {
+  asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %2, 0;\n\t@q st.shared.u16 [%0], %1;\n\t}\n" ::"r"(a),
+               "h"((unsigned short)v), "r"((uint32_t)p)
+               : "memory");
+}
+
 // What one selector thread carries through a tile.
 struct Row {
-  int i, nblk;              // my query block, key blocks
+  int i, nblk, r;           // my query block, key blocks, my row within the item
   bool row;                 // i < nblk
-  float A, B;               // histogram bin map
+  float A, B;               // window bin map
   uint32_t tb;              // the bin being resolved
   float cs;                 // cut: keep s > cs, or s == cs and j <= cj
   int cj;
   uint32_t kpre, kmask, vpre, vmask, sh;  // fallback radix state
   bool vlevel;              // fallback level on the block index bytes
-  uint32_t* hw;             // my 16-bit histogram lane: + bin * 64 words
-  uint32_t inc;
-  float* cand_s;            // my candidate slots: + slot * kRows
-  uint16_t* cand_j;
+  uint32_t h32;             // shared address of my window-histogram column: + bin * 512
+  uint32_t hw;              // shared address of my u16 byte-histogram word: + digit * 256
+  uint32_t inc;             // my half of that word
+  bool bitmask;             // output into the shared bitmask
+  uint32_t mask;            // its shared address
+  uint32_t cs_addr;         // shared address of my candidate scores: + slot * 512
+  uint32_t cj_addr;         // ... and of their block indices: + slot * 256
   int n;                    // candidates found
   int32_t* out;             // my output row
   int w, top;               // kept blocks written; first position of the second warpgroup
@@ -221,11 +275,12 @@ struct Row {
 
 // Output decision for block j with score bits u: the diagonal and every block
 // at or above the cut are written, in my direction.
-SB_DEV void output_one(uint32_t u, int j, bool checks, Row& R) {
-  if (checks && j >= R.nblk) return;
+template <bool Checks>
+SB_DEV void output_one(uint32_t u, int j, Row& R) {
+  if (Checks && j >= R.nblk) return;
   const float s = __uint_as_float(u);
   if (R.srow != nullptr) R.srow[j] = s;
-  const bool kept = (checks && j == R.i) || s > R.cs || (s == R.cs && j <= R.cj);
+  const bool kept = (Checks && j == R.i) || s > R.cs || (s == R.cs && j <= R.cj);
   if (kept) {
     const int pos = R.desc ? R.top - R.w : R.w;
     if (pos >= 0 && pos < R.cap) R.out[pos] = j;  // bounded by the row's capacity
@@ -234,40 +289,40 @@ SB_DEV void output_one(uint32_t u, int j, bool checks, Row& R) {
 }
 
 // One chunk of 32 scores of my row, block indices j0 .. j0+31 (sample pass:
-// sample indices m0 .. m0+31).  `checks`: the tile holds the diagonal or runs
-// past nblk (or is the sample), so each element is tested.
-template <int Kind>
-SB_DEV void scan_chunk(const uint32_t (&v)[32], int j0, bool checks, Row& R) {
+// sample indices j0 .. j0+31).  Checks: the tile holds the diagonal or runs
+// past nblk (or is the sample), so each element is tested; elsewhere the
+// loops have no branch but the rare candidate store.
+template <int Kind, bool Checks>
+SB_DEV void scan_chunk(const uint32_t (&v)[32], int j0, Row& R) {
   if (Kind == kSample) {
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       const int m = j0 + e, j = m * R.stride;
       const float s = __uint_as_float(v[e]);
-      if (m < R.ns && j != R.i) {
-        R.sum += s;
-        R.sq = fmaf(s, s, R.sq);
-        ++R.ns_seen;
-      }
+      const bool use = ((uint32_t)(m < R.ns) & (uint32_t)(j != R.i)) != 0u;
+      R.sum += use ? s : 0.0f;
+      R.sq = fmaf(use ? s : 0.0f, s, R.sq);
+      R.ns_seen += use ? 1 : 0;
     }
   } else if (Kind == kHist) {
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       const int j = j0 + e;
       const uint32_t b = bin_of(__uint_as_float(v[e]), R.A, R.B);
-      if (!checks || (j < R.nblk && j != R.i)) atomicAdd(R.hw + b * 64u, R.inc);
+      const uint32_t valid = Checks ? ((uint32_t)(j < R.nblk) & (uint32_t)(j != R.i)) : 1u;
+      red_add(R.h32 + b * 512u, valid);
     }
   } else if (Kind == kCompact) {
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       const int j = j0 + e;
       const float s = __uint_as_float(v[e]);
-      if (bin_of(s, R.A, R.B) == R.tb && (!checks || (j < R.nblk && j != R.i))) {
-        if (R.n < kCap) {
-          R.cand_s[R.n * kRows] = s;
-          R.cand_j[R.n * kRows] = (uint16_t)j;
-        }
-        ++R.n;
-      }
+      uint32_t take = (uint32_t)(bin_of(s, R.A, R.B) == R.tb);
+      if (Checks) take &= (uint32_t)(j < R.nblk) & (uint32_t)(j != R.i);
+      const bool room = (take & (uint32_t)(R.n < kCap)) != 0u;
+      sts_u32_if(room, R.cs_addr + (uint32_t)R.n * 512u, v[e]);
+      sts_u16_if(room, R.cj_addr + (uint32_t)R.n * 256u, (uint32_t)j);
+      R.n += (int)take;
     }
   } else if (Kind == kLevel) {
 #pragma unroll
@@ -275,17 +330,37 @@ SB_DEV void scan_chunk(const uint32_t (&v)[32], int j0, bool checks, Row& R) {
       const int j = j0 + e;
       const float s = __uint_as_float(v[e]);
       const uint32_t key = order_key(s), vj = 0xFFFFu - (uint32_t)j;
-      const bool member = bin_of(s, R.A, R.B) == R.tb && (key & R.kmask) == R.kpre && (vj & R.vmask) == R.vpre;
+      uint32_t member = (uint32_t)(bin_of(s, R.A, R.B) == R.tb) & (uint32_t)((key & R.kmask) == R.kpre) &
+                        (uint32_t)((vj & R.vmask) == R.vpre);
+      if (Checks) member &= (uint32_t)(j < R.nblk) & (uint32_t)(j != R.i);
       const uint32_t digit = ((R.vlevel ? vj : key) >> R.sh) & 0xFFu;
-      if (member && (!checks || (j < R.nblk && j != R.i))) atomicAdd(R.hw + digit * 64u, R.inc);
+      red_add(R.hw + digit * 256u, member * R.inc);
     }
-  } else {  // kOutput, in my writing direction (constant register indices either way)
+  } else if (R.bitmask) {  // kOutput into the bitmask: one word per chunk
+    uint32_t m = 0;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int j = j0 + e;
+      const float s = __uint_as_float(v[e]);
+      // (bitwise, not short-circuit, so that no lane branches)
+      uint32_t kept = (uint32_t)(s > R.cs) | ((uint32_t)(s == R.cs) & (uint32_t)(j <= R.cj));
+      if (Checks) kept = (kept | (uint32_t)(j == R.i)) & (uint32_t)(j < R.nblk);
+      m |= kept << e;
+    }
+    if (R.srow != nullptr) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (!Checks || j0 + e < R.nblk) R.srow[j0 + e] = __uint_as_float(v[e]);
+    }
+    const uint32_t w = (uint32_t)j0 >> 5;
+    sts_u32(R.mask + (w * kRows + ((uint32_t)R.r ^ (w & 31u))) * 4u, m);
+  } else {  // kOutput written directly, in my direction (constant register indices either way)
     if (R.desc) {
 #pragma unroll
-      for (int e = 31; e >= 0; --e) output_one(v[e], j0 + e, checks, R);
+      for (int e = 31; e >= 0; --e) output_one<Checks>(v[e], j0 + e, R);
     } else {
 #pragma unroll
-      for (int e = 0; e < 32; ++e) output_one(v[e], j0 + e, checks, R);
+      for (int e = 0; e < 32; ++e) output_one<Checks>(v[e], j0 + e, R);
     }
   }
 }
@@ -293,8 +368,8 @@ SB_DEV void scan_chunk(const uint32_t (&v)[32], int j0, bool checks, Row& R) {
 // My 128 columns of accumulator `d` (lane quarter address), in four chunks of
 // 32 with the next chunk's load in flight; descending chunk order for the
 // backward writer.
-template <int Kind>
-SB_DEV void scan_tile(uint32_t d, int jbase, bool checks, Row& R) {
+template <int Kind, bool Checks>
+SB_DEV void scan_tile(uint32_t d, int jbase, Row& R) {
   uint32_t va[32], vb[32];
   const bool back = Kind == kOutput && R.desc;
   tmem_ld_32cols(d + (back ? 96u : 0u), va);
@@ -303,11 +378,19 @@ SB_DEV void scan_tile(uint32_t d, int jbase, bool checks, Row& R) {
     const int ca = back ? 3 - 2 * h : 2 * h, cb = back ? 2 - 2 * h : 2 * h + 1;
     tmem_wait_ld_regs(va);
     tmem_ld_32cols(d + (uint32_t)cb * 32u, vb);
-    if (R.row) scan_chunk<Kind>(va, jbase + ca * 32, checks, R);
+    if (R.row) scan_chunk<Kind, Checks>(va, jbase + ca * 32, R);
     tmem_wait_ld_regs(vb);
     if (h == 0) tmem_ld_32cols(d + (back ? 32u : 64u), va);
-    if (R.row) scan_chunk<Kind>(vb, jbase + cb * 32, checks, R);
+    if (R.row) scan_chunk<Kind, Checks>(vb, jbase + cb * 32, R);
   }
+}
+
+template <int Kind>
+SB_DEV void scan_tile(uint32_t d, int jbase, bool checks, Row& R) {
+  if (checks)
+    scan_tile<Kind, true>(d, jbase, R);
+  else
+    scan_tile<Kind, false>(d, jbase, R);
 }
 
 // Scan my row's 256 bins from the top (clearing them) for the bin where the
@@ -319,20 +402,62 @@ SB_DEV int find_bin(const uint16_t* hist_row, int need, int& above, int& cnt) {
   above = 0;
   cnt = 0;
 #pragma unroll 4
-  for (int b = kBins - 1; b >= 0; --b) {
+  for (int b = kBins - 1; b >= 0; --b) {  // (selects, no branch)
     const int c = h[b * kRows];
     h[b * kRows] = 0;
-    if (bin < 0) {
-      if (cum + c >= need) {
-        bin = b;
-        above = cum;
-        cnt = c;
-      } else {
-        cum += c;
-      }
-    }
+    const bool open = bin < 0;
+    const bool hit = open && cum + c >= need;
+    bin = hit ? b : bin;
+    above = hit ? cum : above;
+    cnt = hit ? c : cnt;
+    cum += (open && !hit) ? c : 0;
   }
   return bin;
+}
+
+// Kept lists of item (bh, rb) from the shared bitmask.  Each of the eight
+// selector warps takes every eighth row, four rows at a time (independent
+// chains: a warp issues only about one instruction every few cycles, so the
+// work per word is kept short and interleaved).  Word by word: lane l keeps
+// block 32 w + l if bit l is set and writes it at the row's running count
+// plus the set bits below l, so a word's kept blocks go out in one store of
+// consecutive entries; then the rows' words are cleared.
+SB_DEV void write_rows(uint8_t* smem, const SelectArgs& a, int bh, int rb, int sel_warp, int lane) {
+  const int W = (a.nblk + 31) >> 5;
+  uint32_t* bm = reinterpret_cast<uint32_t*>(smem + kOffHist);
+  const uint32_t below = (1u << lane) - 1u;
+  for (int r0 = sel_warp; r0 < kRows; r0 += 32) {
+    int32_t* orow[4];
+    int base[4];
+    bool live[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int ii = rb * kRows + r0 + 8 * k;
+      live[k] = ii < a.nblk;
+      orow[k] = a.kept_idx + ((size_t)bh * a.nblk + (live[k] ? ii : 0)) * a.K_capacity;
+      base[k] = 0;
+    }
+#pragma unroll 2
+    for (int w = 0; w < W; ++w) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int rr = r0 + 8 * k;
+        const uint32_t m = live[k] ? bm[w * kRows + (rr ^ (w & 31))] : 0u;  // (every lane reads the same word)
+        const int pos = base[k] + __popc(m & below);
+        stg_s32_if(((m >> lane) & 1u) != 0u && pos < a.K_capacity, orow[k] + pos, w * 32 + lane);
+        base[k] += __popc(m);
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (!live[k]) continue;
+      const int rr = r0 + 8 * k;
+      for (int w = lane; w < W; w += 32) bm[w * kRows + (rr ^ (w & 31))] = 0u;  // zero for the next histogram
+      for (int q = base[k] + lane; q < a.K_capacity; q += 32) orow[k][q] = -1;
+      if (lane == 0) a.kept_cnt[(size_t)bh * a.nblk + rb * kRows + rr] = min(base[k], a.K_capacity);
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -381,148 +506,152 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* plan_slow = &ms->plan_slow;
   const WaitCtl wc{abort_flag, wait_limit_ns};
 
-  if (warp == 0) {
-    // ------------------------------------------------------------- TMA
-    bool ok = true;
-    uint32_t sc = 0, ic = 0;
-    if (lane == 0) {
-      for (int item = blockIdx.x; item < pl.items && ok; item += gridDim.x, ++ic) {
-        const int bh = item / pl.row_blocks;
-        bool slow = false;
-        int total = pl.total(false);
-        for (int p = 0; p < total && ok; ++p) {
-          if (pl.general && p == 3) {
-            if (!(ok = mbar_wait(&ms->plan, ic & 1, wc))) break;
-            slow = *plan_slow != 0;
-            total = pl.total(slow);
-          }
-          const int kind = pl.kind(p, slow), nt = pl.ntiles(kind);
-          for (int pos = 0; pos < nt && ok; ++pos) {
-            const int tile = tile_of(pos, nt);
-            for (int c = 0; c < kChunks && ok; ++c) {
-              const int s = sc % kStages;
-              if (!(ok = mbar_wait(&ms->stage_empty[s], ((sc / kStages) & 1) ^ 1, wc))) break;
-              mbar_arrive_expect_tx(&ms->raw_full[s], kHalfBytes);
-              if (kind == kSample)
-                tma_load_3d(smem + s * kStageBytes, &tm_s, &ms->raw_full[s], c * kChunkD, 0, bh);
-              else
-                tma_load_3d(smem + s * kStageBytes, &tm_k, &ms->raw_full[s], c * kChunkD, tile * kTileN, bh);
-              ++sc;
+  if (warp < 8) {
+    warpgroup_regs_dec<kRegsProducers>();
+    if (warp == 0) {
+      // ------------------------------------------------------------- TMA
+      bool ok = true;
+      uint32_t sc = 0, ic = 0;
+      if (lane == 0) {
+        for (int item = blockIdx.x; item < pl.items && ok; item += gridDim.x, ++ic) {
+          const int bh = item / pl.row_blocks;
+          bool slow = false;
+          int total = pl.total(false);
+          for (int p = 0; p < total && ok; ++p) {
+            if (pl.general && p == 3) {
+              if (!(ok = mbar_wait(&ms->plan, ic & 1, wc))) break;
+              slow = *plan_slow != 0;
+              total = pl.total(slow);
             }
-          }
-        }
-      }
-      if (!ok) {
-        *abort_flag = 1;
-        // copies already issued land before the CTA exits
-        const uint64_t t0 = global_timer_ns();
-        for (int s = 0; s < kStages; ++s) {
-          const uint32_t n_s = (sc + kStages - 1 - s) / kStages;
-          if (n_s > 0)
-            while (!mbar_try_wait(&ms->raw_full[s], (n_s - 1) & 1) && global_timer_ns() - t0 < 100000000ull) {
-            }
-        }
-      }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------- MMA
-    bool ok = true;
-    if (lane == 0) {
-      uint32_t sc = 0, ic = 0, dc0 = 0, dc1 = 0;  // accumulators used so far
-      for (int item = blockIdx.x; item < pl.items && ok; item += gridDim.x, ++ic) {
-        if (!(ok = mbar_wait(&ms->q_ready, ic & 1, wc))) break;
-        bool slow = false;
-        int total = pl.total(false);
-        for (int p = 0; p < total && ok; ++p) {
-          if (pl.general && p == 3) {
-            if (!(ok = mbar_wait(&ms->plan, ic & 1, wc))) break;
-            slow = *plan_slow != 0;
-            total = pl.total(slow);
-          }
-          const int kind = pl.kind(p, slow), nt = pl.ntiles(kind);
-          const bool three = kind != kSample;  // the sample needs hi.hi only
-          for (int pos = 0; pos < nt && ok; ++pos) {
-            const int b = pos & 1;
-            if (!(ok = mbar_wait(&ms->d_empty[b], ((b ? dc1 : dc0) & 1) ^ 1, wc))) break;
-            tc_fence_after();
-            const uint32_t d = tmem + kColD + (uint32_t)b * kTileN;
-            for (int c = 0; c < kChunks && ok; ++c, ++sc) {
-              const int s = sc % kStages;
-              if (!(ok = mbar_wait(&ms->conv_full[s], (sc / kStages) & 1, wc))) break;
-              tc_fence_after();
-              const uint32_t st = smem_addr(smem + s * kStageBytes);
-              const uint64_t bhi0 = smem_desc(st, 16, 1024, kSwizzle128B);
-              const uint64_t blo0 = smem_desc(st + kHalfBytes, 16, 1024, kSwizzle128B);
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t ks = (uint32_t)(c * 4 + kk);  // K-step of 8 channels
-                const uint32_t ahi = tmem + kColQhi + ks * 8, alo = tmem + kColQlo + ks * 8;
-                // +32 bytes per K-step inside the 128-byte row = +2 in the address field
-                const uint64_t bhi = bhi0 + (uint64_t)(kk * 2), blo = blo0 + (uint64_t)(kk * 2);
-                umma_tf32_ts(d, ahi, bhi, (c == 0 && kk == 0) ? 0u : 1u);
-                if (three) {
-                  umma_tf32_ts(d, ahi, blo, 1u);
-                  umma_tf32_ts(d, alo, bhi, 1u);
-                }
+            const int kind = pl.kind(p, slow), nt = pl.ntiles(kind);
+            for (int pos = 0; pos < nt && ok; ++pos) {
+              const int tile = tile_of(pos, nt);
+              for (int c = 0; c < kChunks && ok; ++c) {
+                const int s = sc % kStages;
+                if (!(ok = mbar_wait(&ms->stage_empty[s], ((sc / kStages) & 1) ^ 1, wc))) break;
+                mbar_arrive_expect_tx(&ms->raw_full[s], kHalfBytes);
+                if (kind == kSample)
+                  tma_load_3d(smem + s * kStageBytes, &tm_s, &ms->raw_full[s], c * kChunkD, 0, bh);
+                else
+                  tma_load_3d(smem + s * kStageBytes, &tm_k, &ms->raw_full[s], c * kChunkD, tile * kTileN, bh);
+                ++sc;
               }
-              umma_commit(&ms->stage_empty[s]);
-            }
-            if (ok) {
-              umma_commit(&ms->d_full[b]);
-              (b ? dc1 : dc0) += 1;
             }
           }
         }
-        if (ok) umma_commit(&ms->q_empty);
-      }
-    }
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (lane == 0) {
-      if (!ok) *abort_flag = 1;
-      umma_commit(&ms->drain);  // every MMA of this thread is done before TMEM is freed
-      const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(&ms->drain, 0) && global_timer_ns() - t0 < 100000000ull) {
-      }
-    }
-    __syncwarp();
-  } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------- converters
-    const int tid = threadIdx.x - 128;
-    uint32_t sc = 0, ic = 0;
-    bool ok = true;
-    for (int item = blockIdx.x; item < pl.items && ok; item += gridDim.x, ++ic) {
-      bool slow = false;
-      int total = pl.total(false);
-      for (int p = 0; p < total && ok; ++p) {
-        if (pl.general && p == 3) {
-          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ms->plan, ic & 1, wc)))) break;
-          slow = *plan_slow != 0;
-          total = pl.total(slow);
-        }
-        const int n_stages = pl.ntiles(pl.kind(p, slow)) * kChunks;
-        for (int q = 0; q < n_stages && ok; ++q, ++sc) {
-          const int s = sc % kStages;
-          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ms->raw_full[s], (sc / kStages) & 1, wc)))) break;
-          uint4* hi = reinterpret_cast<uint4*>(smem + s * kStageBytes);
-          uint4* lo = reinterpret_cast<uint4*>(smem + s * kStageBytes + kHalfBytes);
-#pragma unroll 4
-          for (int e = tid; e < kHalfBytes / 16; e += 128) {
-            const uint4 v = hi[e];
-            const uint4 h = make_uint4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
-            hi[e] = h;
-            lo[e] = make_uint4(__float_as_uint(__uint_as_float(v.x) - __uint_as_float(h.x)),
-                               __float_as_uint(__uint_as_float(v.y) - __uint_as_float(h.y)),
-                               __float_as_uint(__uint_as_float(v.z) - __uint_as_float(h.z)),
-                               __float_as_uint(__uint_as_float(v.w) - __uint_as_float(h.w)));
+        if (!ok) {
+          *abort_flag = 1;
+          // copies already issued land before the CTA exits
+          const uint64_t t0 = global_timer_ns();
+          for (int s = 0; s < kStages; ++s) {
+            const uint32_t n_s = (sc + kStages - 1 - s) / kStages;
+            if (n_s > 0)
+              while (!mbar_try_wait(&ms->raw_full[s], (n_s - 1) & 1) && global_timer_ns() - t0 < 100000000ull) {
+              }
           }
-          fence_proxy_async_smem();  // the pieces are read by the tensor core
-          mbar_arrive(&ms->conv_full[s]);
         }
       }
+      __syncwarp();
+    } else if (warp == 1) {
+      // ------------------------------------------------------------- MMA
+      bool ok = true;
+      if (lane == 0) {
+        uint32_t sc = 0, ic = 0, dc0 = 0, dc1 = 0;  // accumulators used so far
+        for (int item = blockIdx.x; item < pl.items && ok; item += gridDim.x, ++ic) {
+          if (!(ok = mbar_wait(&ms->q_ready, ic & 1, wc))) break;
+          bool slow = false;
+          int total = pl.total(false);
+          for (int p = 0; p < total && ok; ++p) {
+            if (pl.general && p == 3) {
+              if (!(ok = mbar_wait(&ms->plan, ic & 1, wc))) break;
+              slow = *plan_slow != 0;
+              total = pl.total(slow);
+            }
+            const int kind = pl.kind(p, slow), nt = pl.ntiles(kind);
+            const bool three = kind != kSample;  // the sample needs hi.hi only
+            for (int pos = 0; pos < nt && ok; ++pos) {
+              const int b = pos & 1;
+              if (!(ok = mbar_wait(&ms->d_empty[b], ((b ? dc1 : dc0) & 1) ^ 1, wc))) break;
+              tc_fence_after();
+              const uint32_t d = tmem + kColD + (uint32_t)b * kTileN;
+              for (int c = 0; c < kChunks && ok; ++c, ++sc) {
+                const int s = sc % kStages;
+                if (!(ok = mbar_wait(&ms->conv_full[s], (sc / kStages) & 1, wc))) break;
+                tc_fence_after();
+                const uint32_t st = smem_addr(smem + s * kStageBytes);
+                const uint64_t bhi0 = smem_desc(st, 16, 1024, kSwizzle128B);
+                const uint64_t blo0 = smem_desc(st + kHalfBytes, 16, 1024, kSwizzle128B);
+  #pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  const uint32_t ks = (uint32_t)(c * 4 + kk);  // K-step of 8 channels
+                  const uint32_t ahi = tmem + kColQhi + ks * 8, alo = tmem + kColQlo + ks * 8;
+                  // +32 bytes per K-step inside the 128-byte row = +2 in the address field
+                  const uint64_t bhi = bhi0 + (uint64_t)(kk * 2), blo = blo0 + (uint64_t)(kk * 2);
+                  umma_tf32_ts(d, ahi, bhi, (c == 0 && kk == 0) ? 0u : 1u);
+                  if (three) {
+                    umma_tf32_ts(d, ahi, blo, 1u);
+                    umma_tf32_ts(d, alo, bhi, 1u);
+                  }
+                }
+                umma_commit(&ms->stage_empty[s]);
+              }
+              if (ok) {
+                umma_commit(&ms->d_full[b]);
+                (b ? dc1 : dc0) += 1;
+              }
+            }
+          }
+          if (ok) umma_commit(&ms->q_empty);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (lane == 0) {
+        if (!ok) *abort_flag = 1;
+        umma_commit(&ms->drain);  // every MMA of this thread is done before TMEM is freed
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(&ms->drain, 0) && global_timer_ns() - t0 < 100000000ull) {
+        }
+      }
+      __syncwarp();
+    } else if (warp >= 4) {
+      // ------------------------------------------------------------- converters
+      const int tid = threadIdx.x - 128;
+      uint32_t sc = 0, ic = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < pl.items && ok; item += gridDim.x, ++ic) {
+        bool slow = false;
+        int total = pl.total(false);
+        for (int p = 0; p < total && ok; ++p) {
+          if (pl.general && p == 3) {
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ms->plan, ic & 1, wc)))) break;
+            slow = *plan_slow != 0;
+            total = pl.total(slow);
+          }
+          const int n_stages = pl.ntiles(pl.kind(p, slow)) * kChunks;
+          for (int q = 0; q < n_stages && ok; ++q, ++sc) {
+            const int s = sc % kStages;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ms->raw_full[s], (sc / kStages) & 1, wc)))) break;
+            uint4* hi = reinterpret_cast<uint4*>(smem + s * kStageBytes);
+            uint4* lo = reinterpret_cast<uint4*>(smem + s * kStageBytes + kHalfBytes);
+  #pragma unroll 4
+            for (int e = tid; e < kHalfBytes / 16; e += 128) {
+              const uint4 v = hi[e];
+              const uint4 h = make_uint4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
+              hi[e] = h;
+              lo[e] = make_uint4(__float_as_uint(__uint_as_float(v.x) - __uint_as_float(h.x)),
+                                 __float_as_uint(__uint_as_float(v.y) - __uint_as_float(h.y)),
+                                 __float_as_uint(__uint_as_float(v.z) - __uint_as_float(h.z)),
+                                 __float_as_uint(__uint_as_float(v.w) - __uint_as_float(h.w)));
+            }
+            fence_proxy_async_smem();  // the pieces are read by the tensor core
+            mbar_arrive(&ms->conv_full[s]);
+          }
+        }
+      }
+      if (!ok && threadIdx.x == 128) *abort_flag = 1;
     }
-    if (!ok && threadIdx.x == 128) *abort_flag = 1;
-  } else if (warp >= 8) {
+  } else {
+    warpgroup_regs_inc<kRegsSelectors>();
     // ------------------------------------------------------------- selectors
     const int wg = (warp - 8) >> 2;
     const int quarter = warp & 3;
@@ -531,10 +660,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint16_t* hist_row = reinterpret_cast<uint16_t*>(smem + kOffHist) + r;  // + bin * kRows
     Row R;
     R.nblk = a.nblk;
-    R.hw = reinterpret_cast<uint32_t*>(smem + kOffHist) + (r >> 1);
+    const uint32_t region = smem_addr(smem + kOffHist);
+    uint32_t* h32 = reinterpret_cast<uint32_t*>(smem + kOffHist) + r;  // my window-histogram column
+    float* cand_s = reinterpret_cast<float*>(smem + kOffHist) + wg * kCap * kRows + r;
+    uint16_t* cand_j = reinterpret_cast<uint16_t*>(smem + kOffCandJ) + wg * kCap * kRows + r;
+    R.h32 = region + (uint32_t)r * 4u;
+    R.hw = region + (uint32_t)(r >> 1) * 4u;
     R.inc = 1u << ((r & 1) * 16);
-    R.cand_s = reinterpret_cast<float*>(smem + kOffHist) + wg * kCap * kRows + r;
-    R.cand_j = reinterpret_cast<uint16_t*>(smem + kOffCandJ) + wg * kCap * kRows + r;
+    R.bitmask = pl.bitmask;
+    R.mask = region;
+    R.r = r;
+    R.cs_addr = smem_addr(cand_s);
+    R.cj_addr = smem_addr(cand_j);
     R.desc = wg == 1;
     R.cap = a.K_capacity;
     R.stride = pl.stride;
@@ -542,6 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // normal quantile of the kept fraction of the off-diagonal blocks
     const float zq = pl.general ? normcdfinvf(1.0f - (float)(a.keep - 1) / (float)(a.nblk - 1)) : 0.0f;
     uint32_t tc = 0, ic = 0;
+    int pend_bh = -1, pend_rb = 0;  // an item whose kept lists wait in the bitmask
     bool ok = true;
     for (int item = blockIdx.x; item < pl.items; item += gridDim.x, ++ic) {
       const int bh = item / pl.row_blocks;
@@ -553,8 +691,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = ok && __all_sync(0xffffffffu, mbar_wait(&ms->q_empty, (ic & 1) ^ 1, wc));
       if (ok) {
         tc_fence_after();
-        const float4* qrow = reinterpret_cast<const float4*>(a.q_bar + ((size_t)bh * a.nblk + (R.row ? R.i : 0)) * kHeadDim) +
-                             wg * 16;
+        const float4* qrow =
+            reinterpret_cast<const float4*>(a.q_bar + ((size_t)bh * a.nblk + (R.row ? R.i : 0)) * kHeadDim) + wg * 16;
 #pragma unroll 1
         for (int part = 0; part < 2; ++part) {
           uint32_t hv[32], lv[32];
@@ -578,6 +716,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&ms->q_ready);
       }
       if (!(ok = sel_and(ok))) break;
+      // ---- the previous item's kept lists, while the tensor core starts on
+      // this item's first tiles
+      if (pend_bh >= 0) {
+        write_rows(smem, a, pend_bh, pend_rb, warp - 8, lane);
+        pend_bh = -1;
+        sel_sync();  // the bitmask is clear before this item writes into it
+      }
       // ---- selection state of my row
       int need = a.keep - 1;  // off-diagonal blocks still to place (budget form)
       if (a.threshold_mode) {
@@ -621,7 +766,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int jbase = tile * kTileN;
           const bool checks = kind == kSample || tile == rb || jbase + kTileN > a.nblk;
           switch (kind) {
-            case kSample: scan_tile<kSample>(d, 0, true, R); break;
+            case kSample: scan_tile<kSample, true>(d, 0, R); break;
             case kHist: scan_tile<kHist>(d, jbase, checks, R); break;
             case kCompact: scan_tile<kCompact>(d, jbase, checks, R); break;
             case kLevel: scan_tile<kLevel>(d, jbase, checks, R); break;
@@ -640,7 +785,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float mean = R.sum / cnt;
               const float sd = sqrtf(fmaxf(R.sq / cnt - mean * mean, 0.0f));
               const float lo = mean + (zq - kWindowSd) * sd;
-              float A = 127.0f / (kWindowSd * sd);  // 254 bins across 2 * kWindowSd * sd
+              float A = (kWinBins - 2) / (2.0f * kWindowSd * sd);  // bins 1 .. 126 across the window
               float B = 1.0f - lo * A;
               if (!(sd > 0.0f) || !isfinite(A) || !isfinite(B)) A = B = 0.0f;  // one bin: the fallback decides
               ms->bin_a[r] = A;
@@ -653,12 +798,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (kind == kHist) {
           bool bad = false;
           if (wg == 0 && R.row) {
-            int above, cnt;
-            const int b = find_bin(hist_row, need, above, cnt);
-            R.tb = b < 0 ? 0u : (uint32_t)b;
+            int cum = 0, tb = -1, above = 0, cnt = 0;
+#pragma unroll 4
+            for (int b = kWinBins - 1; b >= 0; --b) {  // from the top; clears every bin (selects, no branch)
+              const int c = (int)h32[b * kRows];
+              h32[b * kRows] = 0u;
+              const bool open = tb < 0;
+              const bool hit = open && cum + c >= need;
+              tb = hit ? b : tb;
+              above = hit ? cum : above;
+              cnt = hit ? c : cnt;
+              cum += (open && !hit) ? c : 0;
+            }
+            R.tb = tb < 0 ? 0u : (uint32_t)tb;
             need -= above;
-            bad = b < 0 || cnt > kCap;
+            bad = tb < 0 || cnt > kCap;  // (bins 0 and 127, outside the window, are large)
             ms->tb[r] = (int)R.tb;
+            ms->need[r] = need;
           }
           slow = sel_or(bad);
           if (wg == 0 && r == 0) {
@@ -668,45 +824,82 @@ __global__ void __launch_bounds__(kThreads, 1)
           total = pl.total(slow);
           R.tb = (uint32_t)ms->tb[r];
         } else if (kind == kCompact) {
-          if (wg == 1) ms->n1[r] = R.n;
+          // the cut: the candidate with need - 1 candidates before it in
+          // (score descending, index ascending) order; each warpgroup ranks
+          // its own candidates against all of them
+          (wg == 0 ? ms->n0 : ms->n1)[r] = R.n;
+          if (wg == 0) {
+            ms->cut_s[r] = __int_as_float(0x7f800000);  // (none found: nothing but the diagonal)
+            ms->cut_j[r] = -1;
+          }
           sel_sync();
-          if (wg == 0 && R.row) {
-            float* s0 = R.cand_s;                    // my slots, then the second warpgroup's
-            uint16_t* j0 = R.cand_j;
-            float* s1 = R.cand_s + kCap * kRows;
-            uint16_t* j1 = R.cand_j + kCap * kRows;
-            const int n0 = min(R.n, kCap), n1 = min(ms->n1[r], kCap), tot = n0 + n1;
-            R.cs = __int_as_float(0x7f800000);
-            R.cj = -1;
-            for (int x = 0; x < tot; ++x) {
-              const float sx = x < n0 ? s0[x * kRows] : s1[(x - n0) * kRows];
-              const int jx = x < n0 ? j0[x * kRows] : j1[(x - n0) * kRows];
-              int rank = 0;  // candidates before x in (score desc, index asc) order
-              for (int y = 0; y < tot; ++y) {
-                const float sy = y < n0 ? s0[y * kRows] : s1[(y - n0) * kRows];
-                const int jy = y < n0 ? j0[y * kRows] : j1[(y - n0) * kRows];
-                rank += (sy > sx || (sy == sx && jy < jx)) ? 1 : 0;
+          const int n0 = min(ms->n0[r], kCap), n1 = min(ms->n1[r], kCap);
+          float* s0 = cand_s - wg * kCap * kRows;  // the first warpgroup's slots, then the second's
+          uint16_t* j0 = cand_j - wg * kCap * kRows;
+          float* s1 = s0 + kCap * kRows;
+          uint16_t* j1 = j0 + kCap * kRows;
+          if (R.row && n0 + n1 <= 32) {
+            // up to 32 candidates, as 48-bit keys (order key of the score,
+            // then 65535 - index) in registers; each warpgroup ranks 16 slots
+            const int target = ms->need[r] - 1;
+            uint64_t key[32];
+#pragma unroll
+            for (int y = 0; y < 32; ++y) {
+              const bool first = y < n0, second = !first && y - n0 < n1;
+              const int slot = first ? y : y - n0;
+              const float sv = first ? s0[slot * kRows] : (second ? s1[slot * kRows] : 0.0f);
+              const uint32_t jv = first ? j0[slot * kRows] : (second ? j1[slot * kRows] : 0u);
+              key[y] = (first || second) ? (((uint64_t)order_key(sv) << 16) | (uint64_t)(0xFFFFu - jv)) : 0ull;
+            }
+            uint64_t mine[16];  // (selects keep every register index constant)
+            int rank[16];       // independent counts (no chain through one sum)
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+              mine[x] = wg == 0 ? key[x] : key[16 + x];
+              rank[x] = 0;
+            }
+#pragma unroll
+            for (int y = 0; y < 32; ++y)
+#pragma unroll
+              for (int x = 0; x < 16; ++x) rank[x] += key[y] > mine[x] ? 1 : 0;
+#pragma unroll
+            for (int x = 0; x < 16; ++x)
+              if (wg * 16 + x < n0 + n1 && rank[x] == target) {
+                ms->cut_s[r] = key_value((uint32_t)(mine[x] >> 16));
+                ms->cut_j[r] = (int)(0xFFFFu - (uint32_t)(mine[x] & 0xFFFFu));
               }
-              if (rank == need - 1) {
-                R.cs = sx;
-                R.cj = jx;
-                break;
+          } else if (R.row) {
+            // more: each warpgroup ranks its own candidates against all of them
+            const int target = ms->need[r] - 1;
+            const int mine = wg == 0 ? n0 : n1;
+            for (int x = 0; x < mine; ++x) {
+              const float sx = cand_s[x * kRows];
+              const int jx = cand_j[x * kRows];
+              int rank = 0;
+#pragma unroll 4
+              for (int y = 0; y < n0; ++y) {
+                const float sy = s0[y * kRows];
+                rank += (int)((uint32_t)(sy > sx) | ((uint32_t)(sy == sx) & (uint32_t)((int)j0[y * kRows] < jx)));
+              }
+#pragma unroll 4
+              for (int y = 0; y < n1; ++y) {
+                const float sy = s1[y * kRows];
+                rank += (int)((uint32_t)(sy > sx) | ((uint32_t)(sy == sx) & (uint32_t)((int)j1[y * kRows] < jx)));
+              }
+              if (rank == target) {
+                ms->cut_s[r] = sx;
+                ms->cut_j[r] = jx;
               }
             }
-            for (int x = 0; x < n0; ++x) {
-              s0[x * kRows] = 0.0f;
-              j0[x * kRows] = 0;
-            }
-            for (int x = 0; x < n1; ++x) {
-              s1[x * kRows] = 0.0f;
-              j1[x * kRows] = 0;
-            }
-            ms->cut_s[r] = R.cs;
-            ms->cut_j[r] = R.cj;
           }
           sel_sync();
           R.cs = ms->cut_s[r];
           R.cj = ms->cut_j[r];
+          for (int x = 0; x < min(R.n, kCap); ++x) {  // my slots back to zero
+            cand_s[x * kRows] = 0.0f;
+            cand_j[x * kRows] = 0;
+          }
+          sel_sync();  // cleared before the output pass writes the bitmask
         } else if (kind == kLevel) {
           if (wg == 0 && R.row) {
             int above, cnt;
@@ -738,7 +931,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             R.cs = ms->cut_s[r];
             R.cj = ms->cut_j[r];
           }
-        } else {  // kOutput
+        } else if (pl.bitmask) {  // kOutput: the rows are written from the bitmask at the next item's start
+          pend_bh = bh;
+          pend_rb = rb;
+        } else {  // kOutput written directly
           (wg == 0 ? ms->w0 : ms->w1)[r] = R.w;
           sel_sync();
           if (R.row) {
@@ -759,6 +955,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
     }
+    if (ok && pend_bh >= 0) write_rows(smem, a, pend_bh, pend_rb, warp - 8, lane);
     if (!ok) {
       tmem_wait_ld();
       *abort_flag = 1;
@@ -815,6 +1012,10 @@ int launch_select(const SelectArgs& a, cudaStream_t stream) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
     return SBATTN_ERR_CUDA;
+  // the register split (kRegsProducers / kRegsSelectors) adds up to exactly
+  // the launch allocation of 128 per thread; anything else would wait forever
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, select_kernel) != cudaSuccess || fa.numRegs != 128) return SBATTN_ERR_CUDA;
   const long items = (long)a.B * a.H * ((a.nblk + kRows - 1) / kRows);
   const int grid = (int)(items < sms ? items : sms);
   select_kernel<<<grid, kThreads, kSmemBytes, stream>>>(map, sample_map, a, kWaitLimitNs);
