@@ -6,7 +6,9 @@
 // HBM-bound.  Mapping: a CTA owns one 64-token block of one batch and 8 heads
 // (128 "columns" of 16 bytes = 8 channels each); each thread walks the block's
 // tokens in order, so a warp reads and writes 512 contiguous bytes per token
-// (two heads x 256 B) with 128-bit accesses.  The 16 threads of a row reduce
+// (two heads x 256 B) with 128-bit accesses (read-only-path loads and plain
+// write-back stores: faster here than the streaming cache hints), the rows of
+// the next two tokens loaded ahead.  The 16 threads of a row reduce
 // the sum of squares with 4 xor-shuffles.  The (cos, sin) table of every grid
 // position and rotary frequency is built once per CTA in shared memory from
 // fp64 sin/cos; CTAs are persistent over blocks so the table cost is
@@ -21,6 +23,7 @@ namespace {
 
 constexpr int kThreads = 128;       // 8 heads x 16 chunks
 constexpr int kChunks = kHeadDim / 8;  // 16-byte chunks per row
+constexpr int kAhead = 2;              // tokens loaded ahead
 
 SB_DEV void bf16x8_to_f32(const uint4& v, float (&x)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -114,79 +117,83 @@ __global__ void __launch_bounds__(kThreads) prologue_kernel(PrologueArgs a, Rope
       pw = rem - ph * a.W;
     }
 
-    // the rows of the next two tokens are loaded ahead, so that every thread
-    // keeps four 16-byte loads in flight
-    uint4 nq = make_uint4(0, 0, 0, 0), nk = make_uint4(0, 0, 0, 0);
-    uint4 mq = make_uint4(0, 0, 0, 0), mk = make_uint4(0, 0, 0, 0);
-    if (active) {
-      nq = __ldcs(reinterpret_cast<const uint4*>(a.q + base + (size_t)n0 * row_stride));
-      nk = __ldcs(reinterpret_cast<const uint4*>(a.k + base + (size_t)n0 * row_stride));
-      if (n0 + 1 < n1) {
-        mq = __ldcs(reinterpret_cast<const uint4*>(a.q + base + (size_t)(n0 + 1) * row_stride));
-        mk = __ldcs(reinterpret_cast<const uint4*>(a.k + base + (size_t)(n0 + 1) * row_stride));
+    // the rows of the next kAhead tokens are loaded ahead (a ring of kAhead
+    // registers per tensor, indexed by the token's position in the ring, so
+    // the loop is unrolled by kAhead), keeping 2 * kAhead 16-byte loads in
+    // flight per thread
+    uint4 rq[kAhead], rk[kAhead];
+#pragma unroll
+    for (int i = 0; i < kAhead; ++i) {
+      rq[i] = rk[i] = make_uint4(0, 0, 0, 0);
+      if (active && n0 + i < n1) {
+        rq[i] = __ldg(reinterpret_cast<const uint4*>(a.q + base + (size_t)(n0 + i) * row_stride));
+        rk[i] = __ldg(reinterpret_cast<const uint4*>(a.k + base + (size_t)(n0 + i) * row_stride));
       }
     }
-    for (int n = n0; n < n1; ++n) {
-      const size_t off = base + (size_t)n * row_stride;
-      const uint4 vq = nq, vk = nk;
-      nq = mq;
-      nk = mk;
-      if (active && n + 2 < n1) {
-        mq = __ldcs(reinterpret_cast<const uint4*>(a.q + off + 2 * row_stride));
-        mk = __ldcs(reinterpret_cast<const uint4*>(a.k + off + 2 * row_stride));
-      }
-      float xq[8], xk[8];
-      bf16x8_to_f32(vq, xq);
-      bf16x8_to_f32(vk, xk);
-      if constexpr (kNormRope) {
-        float ssq = 0.f, ssk = 0.f;
+    for (int nb = n0; nb < n1; nb += kAhead) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          ssq = fmaf(xq[e], xq[e], ssq);
-          ssk = fmaf(xk[e], xk[e], ssk);
+      for (int i = 0; i < kAhead; ++i) {
+        const int n = nb + i;
+        if (n >= n1) break;  // (the same for every thread of the CTA)
+        const size_t off = base + (size_t)n * row_stride;
+        const uint4 vq = rq[i], vk = rk[i];
+        if (active && n + kAhead < n1) {
+          rq[i] = __ldg(reinterpret_cast<const uint4*>(a.q + off + kAhead * row_stride));
+          rk[i] = __ldg(reinterpret_cast<const uint4*>(a.k + off + kAhead * row_stride));
         }
+        float xq[8], xk[8];
+        bf16x8_to_f32(vq, xq);
+        bf16x8_to_f32(vk, xk);
+        if constexpr (kNormRope) {
+          float ssq = 0.f, ssk = 0.f;
 #pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) {  // the 16 threads of one row
-          ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
-          ssk += __shfl_xor_sync(0xffffffffu, ssk, o);
-        }
-        const float rq = 1.0f / sqrtf(ssq * inv_d + a.eps);
-        const float rk = 1.0f / sqrtf(ssk * inv_d + a.eps);
-        const int pos = axis == 0 ? pt : (axis == 1 ? ph : pw);
-        const float2* cs = tab + rt.off[axis] + pos * rt.half[axis] + m0;
-        uint32_t oq[4], ok[4];
+          for (int e = 0; e < 8; ++e) {
+            ssq = fmaf(xq[e], xq[e], ssq);
+            ssk = fmaf(xk[e], xk[e], ssk);
+          }
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const float2 t = cs[p];
-          float a0 = xq[2 * p] * rq * wq[2 * p], a1 = xq[2 * p + 1] * rq * wq[2 * p + 1];
-          float y0 = a0 * t.x - a1 * t.y, y1 = a0 * t.y + a1 * t.x;
-          oq[p] = pack_bf16x2_rn(y0, y1);
-          a0 = xk[2 * p] * rk * wk[2 * p];
-          a1 = xk[2 * p + 1] * rk * wk[2 * p + 1];
-          y0 = a0 * t.x - a1 * t.y;
-          y1 = a0 * t.y + a1 * t.x;
-          ok[p] = pack_bf16x2_rn(y0, y1);
-        }
-        const uint4 wq4 = make_uint4(oq[0], oq[1], oq[2], oq[3]);
-        const uint4 wk4 = make_uint4(ok[0], ok[1], ok[2], ok[3]);
-        if (active) {
-          __stcs(reinterpret_cast<uint4*>(a.q_out + off), wq4);
-          __stcs(reinterpret_cast<uint4*>(a.k_out + off), wk4);
+          for (int o = 8; o >= 1; o >>= 1) {  // the 16 threads of one row
+            ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
+            ssk += __shfl_xor_sync(0xffffffffu, ssk, o);
+          }
+          const float rq_ = 1.0f / sqrtf(ssq * inv_d + a.eps);
+          const float rk_ = 1.0f / sqrtf(ssk * inv_d + a.eps);
+          const int pos = axis == 0 ? pt : (axis == 1 ? ph : pw);
+          const float2* cs = tab + rt.off[axis] + pos * rt.half[axis] + m0;
+          uint32_t oq[4], ok[4];
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            const float2 t = cs[p];
+            float a0 = xq[2 * p] * rq_ * wq[2 * p], a1 = xq[2 * p + 1] * rq_ * wq[2 * p + 1];
+            float y0 = a0 * t.x - a1 * t.y, y1 = a0 * t.y + a1 * t.x;
+            oq[p] = pack_bf16x2_rn(y0, y1);
+            a0 = xk[2 * p] * rk_ * wk[2 * p];
+            a1 = xk[2 * p + 1] * rk_ * wk[2 * p + 1];
+            y0 = a0 * t.x - a1 * t.y;
+            y1 = a0 * t.y + a1 * t.x;
+            ok[p] = pack_bf16x2_rn(y0, y1);
+          }
+          const uint4 wq4 = make_uint4(oq[0], oq[1], oq[2], oq[3]);
+          const uint4 wk4 = make_uint4(ok[0], ok[1], ok[2], ok[3]);
+          if (active) {
+            *reinterpret_cast<uint4*>(a.q_out + off) = wq4;
+            *reinterpret_cast<uint4*>(a.k_out + off) = wk4;
+          }
+          if constexpr (kPool) {
+            bf16x8_to_f32(wq4, xq);
+            bf16x8_to_f32(wk4, xk);
+          }
+          if (++pw == a.W) {
+            pw = 0;
+            if (++ph == a.Hh) { ph = 0; ++pt; }
+          }
         }
         if constexpr (kPool) {
-          bf16x8_to_f32(wq4, xq);
-          bf16x8_to_f32(wk4, xk);
-        }
-        if (++pw == a.W) {
-          pw = 0;
-          if (++ph == a.Hh) { ph = 0; ++pt; }
-        }
-      }
-      if constexpr (kPool) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          qs[e] += xq[e];
-          ks[e] += xk[e];
+          for (int e = 0; e < 8; ++e) {
+            qs[e] += xq[e];
+            ks[e] += xk[e];
+          }
         }
       }
     }
