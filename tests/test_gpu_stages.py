@@ -173,7 +173,10 @@ def test_threshold_selection_matches_oracle(data):
             expect = [j for j in range(wl.nblk) if j == i or gs[0, h, i, j] >= np.float32(tau)]
             assert got == expect
             assert torch.all(idx[0, h, i, c:] == -1)
-    # and the GPU scores are the oracle's
+    # and the GPU scores are the oracle's (same bound as the budget path)
+    qb, kb = orc.block_pool(qr16), orc.block_pool(kr16)
+    cs = np.linalg.norm(qb, axis=-1)[..., None] * np.max(np.linalg.norm(kb, axis=-1), axis=-1)[..., None, None]
+    assert np.all(np.abs(gs - ref_scores) <= 1e-5 * cs), "threshold-path scores off"
     ref_idx, ref_cnt, _ = orc.select_blocks_threshold(qr16, kr16, tau)
     rows_same = np.mean([set(idx[0, h, i, :cnt[0, h, i]].tolist()) == set(ref_idx[0, h, i, :ref_cnt[0, h, i]].tolist())
                          for h in range(wl.H) for i in range(wl.nblk)])
