@@ -58,19 +58,6 @@ SB_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
-// Non-blocking test of the phase with the given parity (never suspends).
-SB_DEV bool mbar_test(uint64_t* bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-
 // try_wait with a suspend-time hint: the waiting thread sleeps in hardware
 // until the phase completes or about `hint_ns` pass, instead of spinning on
 // issue slots that the other warps of its SM sub-partition need.

@@ -41,6 +41,9 @@
 //   3. compaction: the scores of that bin (a few dozen at most) go to
 //      shared memory with their block index; the (K-1)-th largest under the
 //      order (score descending, block index ascending) among them is the cut;
+//      for nblk <= 2048 this pass also sets the output bitmask of every block
+//      above the bin, and the candidates at or above the cut are added to it
+//      afterwards, so that the output pass is not needed;
 //   4. output: the diagonal and every block at or above the cut.  For nblk
 //      <= 4096 each thread sets one bit per kept block in a shared-memory
 //      bitmask; at the next item's start (while the tensor core begins that
@@ -48,18 +51,21 @@
 //      blocks in one store of consecutive entries.  Beyond 4096 each
 //      warpgroup writes its own tiles' blocks from its end of the row (the
 //      first forward, the second backward from the last position).
-// If some row's bin holds more than 40 blocks (a sample that misplaced the
-// window, or mass ties), the item runs instead six radix levels restricted to
-// that bin: the four bytes of an order-preserving key of the score, then the
-// two bytes of (65535 - block index), which fixes the cut exactly.  Threshold
-// mode (keep s >= tau) and the trivial budgets run the output pass alone.
+// The histogram's counts decide each item's remaining passes: when some
+// row's bin holds more than the merged pass's 20 slots per warpgroup, the
+// item runs compaction (40 slots) and output as separate passes; when some
+// bin holds more than 40 blocks (a sample that misplaced the window, or mass
+// ties), it runs instead six radix levels restricted to that bin: the four
+// bytes of an order-preserving key of the score, then the two bytes of
+// (65535 - block index), which fixes the cut exactly.  Threshold mode (keep
+// s >= tau) and the trivial budgets run the output pass alone.
 //
 // Roles (512 threads, one CTA per SM, persistent over work items):
 //   warp 0: TMA producer           warp 1: TMEM allocator + MMA issuer
 //   warps 4-7: converters          warps 8-15: two selector warpgroups
 //                                  (TMEM lane quarter = warp % 4)
-// The producer warpgroups give up registers (72 per thread) to the selector
-// warpgroups (184), whose chunk code is unrolled over 32 scores.
+// The producer warpgroups give up registers (80 per thread) to the selector
+// warpgroups (176), whose chunk code is unrolled over 32 scores.
 // Every mbarrier wait is bounded; a failed wait is shared with the other
 // selector warpgroup at the next named barrier, after which the kernel stores
 // nothing more, lets its own copies and MMAs finish, frees TMEM and returns.
@@ -81,7 +87,8 @@ constexpr int kStageBytes = 2 * kHalfBytes;
 //   * the window histogram: u32 counts [bin][row], 128 bins (a warp's 32
 //     rows hit 32 banks whatever their bins);
 //   * the candidates of the boundary bin: f32 scores [wg][slot][row], then
-//     u16 block indices [wg][slot][row];
+//     u16 block indices [wg][slot][row] (from 32 KB on, 20 slots, when the
+//     bitmask of a merged compaction-and-output pass holds the first 32 KB);
 //   * the kept-block bitmask: u32 words [word][row ^ (word % 32)], 32 blocks
 //     per word (nblk <= 4096); the xor spreads both a warp's 32 rows of one
 //     word and one row's 32 words over the 32 banks;
@@ -90,9 +97,15 @@ constexpr int kWinBins = 128;
 constexpr int kBins = 256;
 constexpr int kHistBytes = kBins * kRows * 2;         // 64 KB
 constexpr int kOffHist = kStages * kStageBytes;       // 128 KB
-constexpr int kCap = 40;                              // candidates per row and selector warpgroup
-constexpr int kOffCandJ = kOffHist + 2 * kCap * kRows * 4;
-static_assert(kOffCandJ + 2 * kCap * kRows * 2 <= kOffHist + kHistBytes, "candidates fit the shared region");
+// Candidates per row and selector warpgroup: 40 when they have the region to
+// themselves (scores at 0, indices after them), 20 when the merged pass keeps
+// the bitmask in the region's first 32 KB (scores at 32 KB, then indices).
+constexpr int kCap = 40, kCapMerged = 20;
+constexpr int kMergedMaxTiles = 16;                   // bitmask of 64 words per row = 32 KB
+constexpr int kOffCandMerged = 32 * 1024;
+static_assert(2 * kCap * kRows * 6 <= kHistBytes, "candidates fit the shared region");
+static_assert(kOffCandMerged + 2 * kCapMerged * kRows * 6 <= kHistBytes, "merged candidates fit behind the bitmask");
+static_assert(kMergedMaxTiles * 4 * kRows * 4 <= kOffCandMerged, "merged bitmask fits before the candidates");
 static_assert(kWinBins * kRows * 4 <= kHistBytes, "window histogram fits the shared region");
 constexpr int kMaskWords = kHistBytes / (kRows * 4);  // 128 words: 4096 blocks per row
 constexpr int kOffMisc = kOffHist + kHistBytes;       // 192 KB
@@ -101,10 +114,11 @@ constexpr uint32_t kColQhi = 0, kColQlo = 128, kColD = 256;  // accumulator b at
 constexpr int kLevels = 6;                    // fallback: 4 key bytes + 2 index bytes
 constexpr float kWindowSd = 0.75f;            // half-width of the histogram window, in sd
 // registers: the selectors' unrolled chunk code takes the producers' share
-constexpr uint32_t kRegsProducers = 72, kRegsSelectors = 184;
+constexpr uint32_t kRegsProducers = 80, kRegsSelectors = 176;
 static_assert(256 * kRegsProducers + 256 * kRegsSelectors == kThreads * 128, "register split = 512 x 128");
 
-enum PassKind { kSample = 0, kHist = 1, kCompact = 2, kLevel = 3, kOutput = 4 };
+enum PassKind { kSample = 0, kHist = 1, kCompact = 2, kLevel = 3, kOutput = 4, kMerged = 5 };
+enum Verdict { kFast = 0, kSplit = 1, kSlow = 2 };
 
 struct Misc {
   uint64_t raw_full[kStages], conv_full[kStages], stage_empty[kStages];
@@ -197,6 +211,7 @@ struct Plan {
   int items, row_blocks, tiles, stride, ns;
   bool general;  // budget form with 1 < keep < nblk
   bool bitmask;  // kept blocks gathered in shared memory, written row by row
+  bool merged;   // compaction and output in one pass (bitmask and candidates share the region)
   SB_DEV void init(const SelectArgs& a) {
     row_blocks = (a.nblk + kRows - 1) / kRows;
     items = a.B * a.H * row_blocks;
@@ -205,13 +220,21 @@ struct Plan {
     ns = (a.nblk + stride - 1) / stride;
     general = !a.threshold_mode && a.keep > 1 && a.keep < a.nblk;
     bitmask = a.nblk <= kMaskWords * 32;
+    merged = general && tiles <= kMergedMaxTiles;
   }
-  SB_DEV int total(bool slow) const { return general ? (slow ? 3 + kLevels : 4) : 1; }
-  SB_DEV int kind(int p, bool slow) const {
+  // The histogram's verdict on an item: kFast (every boundary bin fits the
+  // candidate slots), kSplit (some bin needs the larger slots of a separate
+  // compaction pass), kSlow (some bin is too large: radix levels).  Passes of
+  // an item; the producers assume four until they read the verdict, before
+  // the fourth.
+  SB_DEV bool merged_for(int v) const { return merged && v == kFast; }
+  SB_DEV int total(int v) const { return general ? (v == kSlow ? 3 + kLevels : (merged_for(v) ? 3 : 4)) : 1; }
+  SB_DEV int total_before_verdict() const { return general ? 4 : 1; }
+  SB_DEV int kind(int p, int v) const {
     if (!general) return kOutput;
     if (p == 0) return kSample;
     if (p == 1) return kHist;
-    if (!slow) return p == 2 ? kCompact : kOutput;
+    if (v != kSlow) return p == 2 ? (merged_for(v) ? kMerged : kCompact) : kOutput;
     return p < 2 + kLevels ? kLevel : kOutput;
   }
   SB_DEV int ntiles(int kind) const { return kind == kSample ? 1 : tiles; }
@@ -223,9 +246,6 @@ SB_DEV int tile_of(int pos, int tiles) { return (pos & 1) ? tiles - 1 - (pos >> 
 // Shared-memory stores and adds on 32-bit shared addresses (no address-space
 // conversion per element); the add returns nothing, so nothing waits for it.
 SB_DEV void sts_u32(uint32_t a, uint32_t v) { asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory"); }
-SB_DEV void sts_u16(uint32_t a, uint32_t v) {
-  asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"((unsigned short)v) : "memory");
-}
 SB_DEV void red_add(uint32_t a, uint32_t v) { asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory"); }
 // Stores under a predicate, with no branch around them (a divergent branch
 // per element costs more than the work it skips).
@@ -262,7 +282,7 @@ struct Row {
   uint32_t mask;            // its shared address
   uint32_t cs_addr;         // shared address of my candidate scores: + slot * 512
   uint32_t cj_addr;         // ... and of their block indices: + slot * 256
-  int n;                    // candidates found
+  int n, cap_slots;         // candidates found, room for them
   int32_t* out;             // my output row
   int w, top;               // kept blocks written; first position of the second warpgroup
   bool desc;                // second warpgroup: writes backwards from top
@@ -319,11 +339,37 @@ SB_DEV void scan_chunk(const uint32_t (&v)[32], int j0, Row& R) {
       const float s = __uint_as_float(v[e]);
       uint32_t take = (uint32_t)(bin_of(s, R.A, R.B) == R.tb);
       if (Checks) take &= (uint32_t)(j < R.nblk) & (uint32_t)(j != R.i);
-      const bool room = (take & (uint32_t)(R.n < kCap)) != 0u;
+      const bool room = (take & (uint32_t)(R.n < R.cap_slots)) != 0u;
       sts_u32_if(room, R.cs_addr + (uint32_t)R.n * 512u, v[e]);
       sts_u16_if(room, R.cj_addr + (uint32_t)R.n * 256u, (uint32_t)j);
       R.n += (int)take;
     }
+  } else if (Kind == kMerged) {
+    // compaction of the boundary bin and the bitmask of the blocks above it
+    // (and the diagonal) in one sweep
+    uint32_t m = 0;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int j = j0 + e;
+      const float s = __uint_as_float(v[e]);
+      const uint32_t b = bin_of(s, R.A, R.B);
+      const uint32_t valid = Checks ? ((uint32_t)(j < R.nblk) & (uint32_t)(j != R.i)) : 1u;
+      const uint32_t take = (uint32_t)(b == R.tb) & valid;
+      const bool room = (take & (uint32_t)(R.n < R.cap_slots)) != 0u;
+      sts_u32_if(room, R.cs_addr + (uint32_t)R.n * 512u, v[e]);
+      sts_u16_if(room, R.cj_addr + (uint32_t)R.n * 256u, (uint32_t)j);
+      R.n += (int)take;
+      uint32_t kept = (uint32_t)(b > R.tb) & valid;
+      if (Checks) kept |= (uint32_t)(j == R.i);
+      m |= kept << e;
+    }
+    if (R.srow != nullptr) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (!Checks || j0 + e < R.nblk) R.srow[j0 + e] = __uint_as_float(v[e]);
+    }
+    const uint32_t w = (uint32_t)j0 >> 5;
+    sts_u32(R.mask + (w * kRows + ((uint32_t)R.r ^ (w & 31u))) * 4u, m);
   } else if (Kind == kLevel) {
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
@@ -515,15 +561,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         for (int item = blockIdx.x; item < pl.items && ok; item += gridDim.x, ++ic) {
           const int bh = item / pl.row_blocks;
-          bool slow = false;
-          int total = pl.total(false);
+          int verdict = kFast;
+          int total = pl.total_before_verdict();
           for (int p = 0; p < total && ok; ++p) {
             if (pl.general && p == 3) {
               if (!(ok = mbar_wait(&ms->plan, ic & 1, wc))) break;
-              slow = *plan_slow != 0;
-              total = pl.total(slow);
+              verdict = *plan_slow;
+              total = pl.total(verdict);
+              if (p >= total) break;
             }
-            const int kind = pl.kind(p, slow), nt = pl.ntiles(kind);
+            const int kind = pl.kind(p, verdict), nt = pl.ntiles(kind);
             for (int pos = 0; pos < nt && ok; ++pos) {
               const int tile = tile_of(pos, nt);
               for (int c = 0; c < kChunks && ok; ++c) {
@@ -559,15 +606,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t sc = 0, ic = 0, dc0 = 0, dc1 = 0;  // accumulators used so far
         for (int item = blockIdx.x; item < pl.items && ok; item += gridDim.x, ++ic) {
           if (!(ok = mbar_wait(&ms->q_ready, ic & 1, wc))) break;
-          bool slow = false;
-          int total = pl.total(false);
+          int verdict = kFast;
+          int total = pl.total_before_verdict();
           for (int p = 0; p < total && ok; ++p) {
             if (pl.general && p == 3) {
               if (!(ok = mbar_wait(&ms->plan, ic & 1, wc))) break;
-              slow = *plan_slow != 0;
-              total = pl.total(slow);
+              verdict = *plan_slow;
+              total = pl.total(verdict);
+              if (p >= total) break;
             }
-            const int kind = pl.kind(p, slow), nt = pl.ntiles(kind);
+            const int kind = pl.kind(p, verdict), nt = pl.ntiles(kind);
             const bool three = kind != kSample;  // the sample needs hi.hi only
             for (int pos = 0; pos < nt && ok; ++pos) {
               const int b = pos & 1;
@@ -619,15 +667,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t sc = 0, ic = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < pl.items && ok; item += gridDim.x, ++ic) {
-        bool slow = false;
-        int total = pl.total(false);
+        int verdict = kFast;
+        int total = pl.total_before_verdict();
         for (int p = 0; p < total && ok; ++p) {
           if (pl.general && p == 3) {
             if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ms->plan, ic & 1, wc)))) break;
-            slow = *plan_slow != 0;
-            total = pl.total(slow);
+            verdict = *plan_slow;
+            total = pl.total(verdict);
+            if (p >= total) break;
           }
-          const int n_stages = pl.ntiles(pl.kind(p, slow)) * kChunks;
+          const int n_stages = pl.ntiles(pl.kind(p, verdict)) * kChunks;
           for (int q = 0; q < n_stages && ok; ++q, ++sc) {
             const int s = sc % kStages;
             if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ms->raw_full[s], (sc / kStages) & 1, wc)))) break;
@@ -662,16 +711,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     R.nblk = a.nblk;
     const uint32_t region = smem_addr(smem + kOffHist);
     uint32_t* h32 = reinterpret_cast<uint32_t*>(smem + kOffHist) + r;  // my window-histogram column
-    float* cand_s = reinterpret_cast<float*>(smem + kOffHist) + wg * kCap * kRows + r;
-    uint16_t* cand_j = reinterpret_cast<uint16_t*>(smem + kOffCandJ) + wg * kCap * kRows + r;
+    // candidate slots: their layout follows each item's verdict
+    int cap = kCap;
+    float* cand_s = nullptr;
+    uint16_t* cand_j = nullptr;
+    auto place_candidates = [&](bool merged_item) {
+      cap = merged_item ? kCapMerged : kCap;
+      float* base = reinterpret_cast<float*>(smem + kOffHist + (merged_item ? kOffCandMerged : 0));
+      cand_s = base + wg * cap * kRows + r;
+      cand_j = reinterpret_cast<uint16_t*>(base + 2 * cap * kRows) + wg * cap * kRows + r;
+      R.cs_addr = smem_addr(cand_s);
+      R.cj_addr = smem_addr(cand_j);
+      R.cap_slots = cap;
+    };
     R.h32 = region + (uint32_t)r * 4u;
     R.hw = region + (uint32_t)(r >> 1) * 4u;
     R.inc = 1u << ((r & 1) * 16);
     R.bitmask = pl.bitmask;
     R.mask = region;
     R.r = r;
-    R.cs_addr = smem_addr(cand_s);
-    R.cj_addr = smem_addr(cand_j);
+    place_candidates(pl.merged);
     R.desc = wg == 1;
     R.cap = a.K_capacity;
     R.stride = pl.stride;
@@ -748,10 +807,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       R.srow = a.scores != nullptr && R.row ? a.scores + ((size_t)bh * a.nblk + R.i) * a.nblk : nullptr;
       R.sum = R.sq = 0.0f;
       R.ns_seen = 0;
-      bool slow = false;
-      int total = pl.total(false);
+      int verdict = kFast;
+      int total = pl.total(kFast);
       for (int p = 0; p < total; ++p) {
-        const int kind = pl.kind(p, slow), nt = pl.ntiles(kind);
+        const int kind = pl.kind(p, verdict), nt = pl.ntiles(kind);
         const int mine = wg == 0 ? (nt + 1) / 2 : nt / 2;
         if (kind == kLevel) {
           const int lvl = p - 2;
@@ -769,6 +828,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             case kSample: scan_tile<kSample, true>(d, 0, R); break;
             case kHist: scan_tile<kHist>(d, jbase, checks, R); break;
             case kCompact: scan_tile<kCompact>(d, jbase, checks, R); break;
+            case kMerged: scan_tile<kMerged>(d, jbase, checks, R); break;
             case kLevel: scan_tile<kLevel>(d, jbase, checks, R); break;
             default: scan_tile<kOutput>(d, jbase, checks, R); break;
           }
@@ -796,7 +856,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           R.A = ms->bin_a[r];
           R.B = ms->bin_b[r];
         } else if (kind == kHist) {
-          bool bad = false;
+          bool bad = false, big = false;
           if (wg == 0 && R.row) {
             int cum = 0, tb = -1, above = 0, cnt = 0;
 #pragma unroll 4
@@ -813,17 +873,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             R.tb = tb < 0 ? 0u : (uint32_t)tb;
             need -= above;
             bad = tb < 0 || cnt > kCap;  // (bins 0 and 127, outside the window, are large)
+            big = cnt > kCapMerged;
             ms->tb[r] = (int)R.tb;
             ms->need[r] = need;
           }
-          slow = sel_or(bad);
+          const bool slow_item = sel_or(bad);
+          const bool split_item = sel_or(big);
+          verdict = slow_item ? kSlow : (split_item ? kSplit : kFast);
           if (wg == 0 && r == 0) {
-            *plan_slow = slow ? 1 : 0;
+            *plan_slow = verdict;
             mbar_arrive(&ms->plan);
           }
-          total = pl.total(slow);
+          total = pl.total(verdict);
+          place_candidates(pl.merged_for(verdict));
           R.tb = (uint32_t)ms->tb[r];
-        } else if (kind == kCompact) {
+        } else if (kind == kCompact || kind == kMerged) {
           // the cut: the candidate with need - 1 candidates before it in
           // (score descending, index ascending) order; each warpgroup ranks
           // its own candidates against all of them
@@ -833,11 +897,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             ms->cut_j[r] = -1;
           }
           sel_sync();
-          const int n0 = min(ms->n0[r], kCap), n1 = min(ms->n1[r], kCap);
-          float* s0 = cand_s - wg * kCap * kRows;  // the first warpgroup's slots, then the second's
-          uint16_t* j0 = cand_j - wg * kCap * kRows;
-          float* s1 = s0 + kCap * kRows;
-          uint16_t* j1 = j0 + kCap * kRows;
+          const int n0 = min(ms->n0[r], cap), n1 = min(ms->n1[r], cap);
+          float* s0 = cand_s - wg * cap * kRows;  // the first warpgroup's slots, then the second's
+          uint16_t* j0 = cand_j - wg * cap * kRows;
+          float* s1 = s0 + cap * kRows;
+          uint16_t* j1 = j0 + cap * kRows;
           if (R.row && n0 + n1 <= 32) {
             // up to 32 candidates, as 48-bit keys (order key of the score,
             // then 65535 - index) in registers; each warpgroup ranks 16 slots
@@ -895,11 +959,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           sel_sync();
           R.cs = ms->cut_s[r];
           R.cj = ms->cut_j[r];
-          for (int x = 0; x < min(R.n, kCap); ++x) {  // my slots back to zero
+          if (kind == kMerged && R.row) {
+            // the candidates at or above the cut join the bitmask
+            uint32_t* bm = reinterpret_cast<uint32_t*>(smem + kOffHist);
+            for (int x = 0; x < min(R.n, cap); ++x) {
+              const float sx = cand_s[x * kRows];
+              const uint32_t jx = cand_j[x * kRows];
+              if (sx > R.cs || (sx == R.cs && (int)jx <= R.cj)) {
+                const uint32_t w = jx >> 5;
+                atomicOr(bm + w * kRows + ((uint32_t)r ^ (w & 31u)), 1u << (jx & 31u));
+              }
+            }
+          }
+          for (int x = 0; x < min(R.n, cap); ++x) {  // my slots back to zero
             cand_s[x * kRows] = 0.0f;
             cand_j[x * kRows] = 0;
           }
           sel_sync();  // cleared before the output pass writes the bitmask
+          if (kind == kMerged) {  // the rows are written from the bitmask at the next item's start
+            pend_bh = bh;
+            pend_rb = rb;
+          }
         } else if (kind == kLevel) {
           if (wg == 0 && R.row) {
             int above, cnt;

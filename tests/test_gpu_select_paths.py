@@ -13,7 +13,10 @@ compared with the oracle's selection on the same pooled means:
   * twin blocks: every score appears twice, so the boundary bin holds exact
     ties that the cut resolves by block index (fast path);
   * several tiles per row in threshold mode, where the second selector
-    warpgroup's blocks are moved behind the first's, and the trivial budgets.
+    warpgroup's blocks are moved behind the first's, and the trivial budgets;
+  * long rows: up to 16 tiles compaction and output share one pass, beyond
+    that they are two passes, and beyond 4096 blocks the rows are written
+    without the shared bitmask.
 """
 
 import numpy as np
@@ -140,3 +143,18 @@ def test_trivial_budgets_over_several_tiles():
     assert torch.all(cnt == 1)
     assert torch.equal(idx[..., 0].cpu(), torch.arange(nblk, dtype=torch.int32).expand(B, H, nblk))
     assert torch.all(idx[..., 1:] == -1)
+
+
+@pytest.mark.parametrize("nblk", [2100, 4200])
+def test_long_rows_take_the_two_pass_and_direct_output_forms(nblk):
+    """Rows of more than 16 tiles run compaction and output as two passes
+    (2100 blocks: 17 tiles, the kept blocks still gathered in the bitmask);
+    beyond 4096 blocks the bitmask does not fit and each warpgroup writes its
+    tiles' blocks itself (4200 blocks)."""
+    rng = np.random.default_rng(55 + nblk)
+    B, H, d = 1, 1, 128
+    u = rng.normal(size=(B, H, nblk, d))
+    q_bar = (rng.normal(size=(B, H, nblk, d)) + 0.5 * u).astype(np.float32).astype(np.float64)
+    k_bar = (rng.normal(size=(B, H, nblk, d)) + 0.5 * u).astype(np.float32).astype(np.float64)
+    stats, gidx, ref_idx = _check_budget(q_bar, k_bar, 0.75)
+    assert stats["decision_agreement"] > 0.9999
