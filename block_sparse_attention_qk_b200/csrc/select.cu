@@ -27,7 +27,8 @@
 //   * The tiles of a pass alternate between the two selector warpgroups: the
 //     first takes tiles 0, 1, 2, ... (accumulator 0), the second tiles T-1,
 //     T-2, ... (accumulator 1).
-// Exact top-K per row, in four passes over the scores:
+// Exact top-K per row, in up to four passes over the scores (three when
+// compaction and output merge):
 //   1. sample: one tile of every ceil(nblk/128)-th key block, one product
 //      (hi.hi); mean m and deviation sd of the row's sampled scores place a
 //      window of 1.5 sd around m + z sd, z the normal quantile of the kept
@@ -124,11 +125,11 @@ struct Misc {
   uint64_t raw_full[kStages], conv_full[kStages], stage_empty[kStages];
   uint64_t d_full[2], d_empty[2];  // accumulator b belongs to selector warpgroup b
   uint64_t q_ready, q_empty;       // the item's Q pieces in TMEM
-  uint64_t plan;                   // one phase per item: fast or fallback schedule
+  uint64_t plan;                   // one phase per item: its verdict is in plan_verdict
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
-  int plan_slow;
+  int plan_verdict;
   // per query block of the item, written by the first selector warpgroup
   float bin_a[kRows], bin_b[kRows], cut_s[kRows];
   int cut_j[kRows], tb[kRows];
@@ -531,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&ms->plan, 1);
     mbar_init(&ms->drain, 1);
     ms->abort = 0;
-    ms->plan_slow = 0;
+    ms->plan_verdict = 0;
     fence_barrier_init();
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_s);
@@ -549,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ms->tmem_base;
   volatile int* abort_flag = &ms->abort;
-  volatile int* plan_slow = &ms->plan_slow;
+  volatile int* plan_verdict = &ms->plan_verdict;
   const WaitCtl wc{abort_flag, wait_limit_ns};
 
   if (warp < 8) {
@@ -566,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int p = 0; p < total && ok; ++p) {
             if (pl.general && p == 3) {
               if (!(ok = mbar_wait(&ms->plan, ic & 1, wc))) break;
-              verdict = *plan_slow;
+              verdict = *plan_verdict;
               total = pl.total(verdict);
               if (p >= total) break;
             }
@@ -611,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int p = 0; p < total && ok; ++p) {
             if (pl.general && p == 3) {
               if (!(ok = mbar_wait(&ms->plan, ic & 1, wc))) break;
-              verdict = *plan_slow;
+              verdict = *plan_verdict;
               total = pl.total(verdict);
               if (p >= total) break;
             }
@@ -672,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int p = 0; p < total && ok; ++p) {
           if (pl.general && p == 3) {
             if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ms->plan, ic & 1, wc)))) break;
-            verdict = *plan_slow;
+            verdict = *plan_verdict;
             total = pl.total(verdict);
             if (p >= total) break;
           }
@@ -881,7 +882,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool split_item = sel_or(big);
           verdict = slow_item ? kSlow : (split_item ? kSplit : kFast);
           if (wg == 0 && r == 0) {
-            *plan_slow = verdict;
+            *plan_verdict = verdict;
             mbar_arrive(&ms->plan);
           }
           total = pl.total(verdict);
