@@ -135,7 +135,10 @@ SBATTN_API size_t sbattn_select_workspace_bytes(int B, int N, int H, int d);
 
 /* For every (b, h) and query block i:
  *   q_bar_i = mean of the (up to) 64 rows of q_rot in block i (k_bar likewise);
- *   score s_ij = q_bar_i . k_bar_j  (fp32);
+ *   score s_ij = q_bar_i . k_bar_j  (fp32; computed on the tensor cores from
+ *   tf32 pieces of each operand, three products, within a few 1e-6 of
+ *   |q_bar_i| |k_bar_j| of the exact dot product; the selection below is
+ *   exact on these scores);
  *   kept(i) = {i} + the K-1 highest-scoring j != i (equal scores: lower j
  *   first), written sorted ascending.
  *
